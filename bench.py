@@ -1,0 +1,449 @@
+"""Batch-256 SSM-layer decode throughput of the ReplaySSM path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--layer mamba2|gdn]
+                    [--impl rssm|reference]
+
+One *step* is one full window of the layer: L = 16 decode calls for every
+sequence of the batch (256 sequences per GPU), the last of which folds the
+window into the fp32 checkpoint; so a step decodes 256 x 16 tokens per GPU
+and every timed step moves the same bytes.  The timed region starts with the
+checkpoint, the ring buffers and a pool of 32 seeded synthetic tokens already
+resident in HBM; the 1 GiB (Mamba-2) / 512 MiB (GDN) checkpoint is far larger
+than the 126 MB L2, so no L2 flush is needed between steps.
+
+Multi-GPU: each rank decodes its own independent batch of 256 sequences
+(replicas; the decode path has no exchange step), value = all ranks' tokens
+divided by the slowest rank's device time.
+
+Reported beside the headline: the conventional per-token update kernel on the
+same layer and inputs (in-run baseline), the end-to-end rate through the C ABI
+with host-resident inputs and outputs, the roofline of the replay kernel, and
+the fp64 CPU oracle timed on this host.  ``--impl reference`` times only the
+oracle (rank 0) and prints its own line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+POOL = 32
+
+
+# ------------------------------------------------------------------ helpers
+def dist_setup(ngpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != ngpus:
+        raise SystemExit(f"--gpus {ngpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML in a thread."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, dev_index, period=0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(pynvml, dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reason_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # no NVML: report it rather than guess
+            self.err = str(e)
+
+    @staticmethod
+    def _handle(pynvml, dev_index):
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[dev_index]) if vis and vis.split(",")[0].isdigit() else dev_index
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self._reason_fn(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, files):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+    except Exception:
+        return None
+    return rec["bytes_per_launch"] if rec.get("source_hash") == source_hash(files) else None
+
+
+# -------------------------------------------------------------- workloads
+class Mamba2Work:
+    name = "mamba2"
+    keys = ("x", "B", "C", "dt")
+    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/mamba2.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
+
+    def __init__(self, dev, seed, batch=None):
+        from hybrid_ssm_decode_replayssm_b200 import rssm
+        self.shape = s = si.MAMBA2_SERVING if batch is None else si.MAMBA2_SERVING.with_(batch=batch)
+        A, D = si.mamba2_params(s, seed)
+        self.A, self.D = A.to(dev), D.to(dev)
+        self.h0 = si.mamba2_checkpoint(s, seed).to(dev)
+        self.desc = rssm.make_desc(rssm.RSSM_MAMBA2, s.batch, s.nheads, s.headdim, s.dstate,
+                                   ngroups=s.ngroups, window=s.window, max_draft=s.max_draft,
+                                   in_dtype=rssm.RSSM_BF16)
+        self.host_pool = [si.mamba2_tokens(s, t, seed) for t in range(POOL)]
+        self.pool = [[tok[k].to(dev) for k in self.keys] for tok in self.host_pool]
+        self.out_shape = (s.batch, s.nheads, s.headdim)
+        self.tokens_per_call = s.batch
+        self.workload = (f"Mamba-2 decode layer: batch {s.batch}, {s.nheads} heads, headdim {s.headdim}, "
+                         f"dstate {s.dstate}, {s.ngroups} groups, bf16 x/B/C/dt, fp32 checkpoint, L={s.window}")
+
+    def layer(self):
+        from hybrid_ssm_decode_replayssm_b200 import rssm
+        return rssm.ReplayLayer(self.desc, self.h0.clone(), self.A, self.D)
+
+    def bytes_per_call(self, pos):
+        """Algorithmic bytes of the decode call at window position pos (1..L)."""
+        s = self.shape
+        B, H, P, N, G, L = s.batch, s.nheads, s.headdim, s.dstate, s.ngroups, s.window
+        e = 2
+        ck = B * H * P * N * 4
+        inp = B * H * P * e + 2 * B * G * N * e + B * H * e
+        entry = B * H * P * e + B * G * N * e + B * H * 4
+        out = B * H * P * 4
+        return ck + inp + entry + (pos - 1) * entry + out + (ck if pos == L else 0)
+
+    def conventional_bytes(self):
+        s = self.shape
+        B, H, P, N, G = s.batch, s.nheads, s.headdim, s.dstate, s.ngroups
+        return 2 * B * H * P * N * 4 + B * H * P * 2 + 2 * B * G * N * 2 + B * H * 2 + B * H * P * 4
+
+    def oracle_sample(self, nseq, steps, seed):
+        """Time the fp64 oracle (conventional recurrence) on nseq sequences x all heads."""
+        from oracle import mamba2 as om
+        h = self.h0[:nseq].double().cpu().numpy()
+        A = self.A.double().cpu().numpy()
+        D = self.D.double().cpu().numpy()
+        toks = [{k: v[:nseq].double().numpy() for k, v in self.host_pool[t % POOL].items()} for t in range(steps)]
+        t0 = time.perf_counter()
+        for tok in toks:
+            h, _ = om.step(h, tok["x"], tok["B"], tok["C"], tok["dt"], A, D)
+        return time.perf_counter() - t0
+
+
+WORKLOADS = {"mamba2": Mamba2Work}
+
+
+# ------------------------------------------------------------------ timing
+def time_replay(work, layer, steps, warmup, L, out, dev, world, sampler_dev):
+    """Device-time `steps` windows of L decode calls; per-launch events too."""
+    from hybrid_ssm_decode_replayssm_b200 import rssm
+    stream = torch.cuda.current_stream()
+    t = 0
+    for _ in range(warmup * L):
+        layer.decode_step(work.pool[t % POOL], out)
+        t += 1
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps * L)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = rssm.lib().rssm_launch_count()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(sampler_dev) as clk:
+        start.record(stream)
+        for i in range(steps * L):
+            ev[i][0].record(stream)
+            layer.decode_step(work.pool[t % POOL], out)
+            ev[i][1].record(stream)
+            t += 1
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches = rssm.lib().rssm_launch_count() - launches0
+    elapsed = start.elapsed_time(stop) / 1e3
+    per = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    positions = [((warmup * L + i) % L) + 1 for i in range(steps * L)]
+    return elapsed, per, positions, launches, clk.summary()
+
+
+def time_conventional(work, layer, steps, warmup, L, out, world):
+    state = work.h0.clone()
+    t = 0
+    for _ in range(warmup * L):
+        layer.conventional_step(state, state, work.pool[t % POOL], out)
+        t += 1
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    start.record()
+    for _ in range(steps * L):
+        layer.conventional_step(state, state, work.pool[t % POOL], out)
+        t += 1
+    stop.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(stop) / 1e3
+
+
+def time_e2e(work, layer, steps, warmup, L, dev, world):
+    """Inputs copied host->device from pinned memory and outputs copied back every
+    call, pipelined on separate copy streams, through the C-ABI decode call."""
+    host_in = [[t.pin_memory() for t in (tok[k] for k in work.keys)] for tok in work.host_pool]
+    nslot = 4
+    dev_in = [[torch.empty_like(t, device=dev) for t in host_in[0]] for _ in range(nslot)]
+    dev_out = [torch.empty(work.out_shape, device=dev) for _ in range(nslot)]
+    host_out = [torch.empty(work.out_shape).pin_memory() for _ in range(nslot)]
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    comp = torch.cuda.current_stream()
+    ev_in = [torch.cuda.Event() for _ in range(nslot)]
+    ev_done = [torch.cuda.Event() for _ in range(nslot)]
+    ev_out = [torch.cuda.Event() for _ in range(nslot)]
+    for e in ev_out:
+        e.record(s_d2h)
+    in_bytes = sum(t.numel() * t.element_size() for t in host_in[0])
+    out_bytes = dev_out[0].numel() * 4
+
+    def run(ncalls, t0):
+        for i in range(ncalls):
+            slot, t = i % nslot, t0 + i
+            with torch.cuda.stream(s_h2d):
+                s_h2d.wait_event(ev_done[slot])          # slot's inputs no longer read
+                for d, h in zip(dev_in[slot], host_in[t % POOL]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[slot].record(s_h2d)
+            comp.wait_event(ev_in[slot])
+            comp.wait_event(ev_out[slot])                # slot's previous output copied out
+            layer.decode_step(dev_in[slot], dev_out[slot], stream=comp)
+            ev_done[slot].record(comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_done[slot])
+                host_out[slot].copy_(dev_out[slot], non_blocking=True)
+                ev_out[slot].record(s_d2h)
+        return t0 + ncalls
+
+    t = run(warmup * L, 0)
+    torch.cuda.synchronize()
+    barrier(world)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(comp)
+    run(steps * L, t)
+    comp.wait_stream(s_d2h)
+    comp.wait_stream(s_h2d)
+    stop.record(comp)
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(stop) / 1e3, in_bytes * L, out_bytes * L
+
+
+def cpu_baseline(work, seed, budget_s=12.0):
+    """The fp64 oracle as it stands, single-threaded (BLAS pinned to 1 thread)."""
+    from threadpoolctl import threadpool_limits
+    nseq = 8
+    with threadpool_limits(1):
+        t1 = work.oracle_sample(nseq, 1, seed)
+        steps = max(2, min(64, int(budget_s / max(t1, 1e-3))))
+        el = work.oracle_sample(nseq, steps, seed)
+    return {"value": nseq * steps / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{nseq} of {work.shape.batch} sequences (all {work.shape.nheads} heads), "
+                       f"{steps} decode steps of the fp64 numpy recurrence, 1 thread"),
+            "seconds": round(el, 2)}
+
+
+# -------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--layer", default="mamba2", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch (profiling captures only; the metric is quoted at 256)")
+    ap.add_argument("--legs", default="replay,conventional,e2e",
+                    help="comma list of timed legs (profiling captures run 'replay' alone)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    seed = args.seed + rank
+    work = WORKLOADS[args.layer](dev, seed, args.batch)
+    legs = set(args.legs.split(","))
+    L = work.shape.window
+    tokens_per_step = work.tokens_per_call * L
+    cfg = {"workload": work.workload, "global_batch": work.shape.batch * world,
+           "tokens_per_step": tokens_per_step * world,
+           "step": f"one window: {L} decode calls per sequence, the last folding the window",
+           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+           "l2": "no flush: the fp32 checkpoint (>= 512 MiB) is larger than L2 and streamed every call"}
+
+    if args.impl == "reference":
+        if rank == 0:
+            cb = cpu_baseline(work, seed, budget_s=max(5.0, 2.0 * args.steps / 10))
+            line = {"impl": "reference", "metric": "SSM-layer decode tokens/s at batch 256",
+                    "value": cb["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                    "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "config": cfg,
+                    "cpu_baseline": cb,
+                    "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    layer = work.layer()
+    out = torch.empty(work.out_shape, device=dev)
+    elapsed, per, positions, launches, clocks = time_replay(work, layer, args.steps, args.warmup, L,
+                                                            out, dev, world, local)
+    elapsed = max_over_ranks(elapsed, world, dev)
+    value = world * tokens_per_step * args.steps / elapsed
+
+    alg_bytes = sum(work.bytes_per_call(p) for p in positions)
+    kern_time = sum(per)
+    peak, peak_kind = measured_peak()
+    achieved = alg_bytes / kern_time / 1e9
+    traffic = ncu_traffic(f"{work.name}_decode", work.kernel_files)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} copy bandwidth",
+                "kernel": f"{work.name} replay decode (append + output, fold every {L}th call)",
+                "bytes_per_launch_avg": alg_bytes / len(per),
+                "launch_us_avg": round(kern_time / len(per) * 1e6, 2)}
+
+    conv = None
+    if "conventional" in legs:
+        conv_el = time_conventional(work, layer, args.steps, args.warmup, L, out, world)
+        conv_el = max_over_ranks(conv_el, world, dev)
+        conv_value = world * tokens_per_step * args.steps / conv_el
+        conv = {"value": round(conv_value, 1), "unit": "tokens/s",
+                "hbm_gbs": round(work.conventional_bytes() * L * args.steps / conv_el / 1e9 * world, 1),
+                "replay_speedup": round(value / conv_value, 3)}
+
+    e2e = None
+    if "e2e" in legs:
+        e2e_layer = work.layer()
+        e2e_el, h2d, d2h = time_e2e(work, e2e_layer, args.steps, args.warmup, L, dev, world)
+        e2e_el = max_over_ranks(e2e_el, world, dev)
+        e2e = {"value": round(world * tokens_per_step * args.steps / e2e_el, 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "how": "rssm_decode_step per call with pinned-host inputs copied in and outputs "
+                      "copied out, pipelined on copy streams"}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(work, seed)
+
+    if rank == 0:
+        line = {"metric": "SSM-layer decode tokens/s at batch 256", "value": round(value, 1),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded; bf16 inputs, fp32 checkpoint)", "config": cfg,
+                "hbm_gbs": round(alg_bytes / elapsed / 1e9 * world, 1),
+                "roofline": roofline, "clocks": clocks, "gpu_launches": int(launches),
+                "e2e": e2e, "conventional": conv,
+                "cpu_baseline": cb}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

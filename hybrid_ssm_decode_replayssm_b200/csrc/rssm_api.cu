@@ -1,0 +1,343 @@
+// Host side of the librssm C ABI: argument checks, buffer layout, launches.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "rssm_internal.h"
+
+struct rssm_handle {
+  rssm_layer_desc d;
+  rssm_layout lay;
+  size_t ckpt_bytes, buf_bytes, rc_bytes, meta_bytes;
+  float *ckpt;
+  uint8_t *buf, *rc, *meta;
+  const float *A, *D;
+};
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<uint64_t> g_launches{0};
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+  char msg[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(msg, sizeof msg, fmt, ap);
+  va_end(ap);
+  g_err = msg;
+  return code;
+}
+
+int ok() {
+  g_err.clear();
+  return RSSM_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+  return fail(RSSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int validate_desc(const rssm_layer_desc *d) {
+  if (!d) return fail(RSSM_ERR_INVALID_ARG, "desc is NULL");
+  if (d->kind != RSSM_MAMBA2 && d->kind != RSSM_GDN)
+    return fail(RSSM_ERR_INVALID_ARG, "kind must be RSSM_MAMBA2 or RSSM_GDN");
+  if (d->batch < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1)
+    return fail(RSSM_ERR_INVALID_ARG, "batch, nheads, headdim and dstate must be positive");
+  if ((long long)d->batch * d->nheads > (1LL << 31) - 1)
+    return fail(RSSM_ERR_INVALID_ARG, "batch * nheads too large");
+  if (d->kind == RSSM_MAMBA2 && (d->ngroups < 1 || d->nheads % d->ngroups))
+    return fail(RSSM_ERR_INVALID_ARG, "nheads must be a positive multiple of ngroups");
+  if (d->window < 1 || d->window > rssm::kMaxWindow)
+    return fail(RSSM_ERR_INVALID_ARG, "window must be in [1, %d]", rssm::kMaxWindow);
+  if (d->max_draft < 0 || d->max_draft > rssm::kMaxDraft || d->max_draft > d->window)
+    return fail(RSSM_ERR_INVALID_ARG, "max_draft must be in [0, min(window, %d)]", rssm::kMaxDraft);
+  if (d->in_dtype != RSSM_F32 && d->in_dtype != RSSM_BF16)
+    return fail(RSSM_ERR_INVALID_ARG, "in_dtype must be RSSM_F32 or RSSM_BF16");
+  if (d->read_fmt != RSSM_READ_FP32 && d->read_fmt != RSSM_READ_FP8_E4M3_ROW &&
+      d->read_fmt != RSSM_READ_NVFP4)
+    return fail(RSSM_ERR_INVALID_ARG, "unknown read_fmt");
+  const bool sup = d->kind == RSSM_MAMBA2 ? rssm::mamba2_supported(d->headdim, d->dstate)
+                                          : rssm::gdn_supported(d->headdim, d->dstate);
+  if (!sup)
+    return fail(RSSM_ERR_UNSUPPORTED, "no kernel for %s headdim=%d dstate=%d in this build",
+                d->kind == RSSM_MAMBA2 ? "Mamba-2" : "GDN", d->headdim, d->dstate);
+  return RSSM_OK;
+}
+
+void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size_t *buf,
+                    size_t *rc, size_t *meta) {
+  std::memset(L, 0, sizeof *L);
+  const size_t B = d->batch, H = d->nheads, R = d->headdim, C = d->dstate;
+  const size_t cap = d->window + (d->max_draft > 1 ? d->max_draft : 1);
+  const size_t esz = d->in_dtype == RSSM_BF16 ? 2 : 4;
+  L->cap = cap;
+  *ckpt = B * H * R * C * sizeof(float);
+  size_t off = 0;
+  if (d->kind == RSSM_MAMBA2) {
+    const size_t G = d->ngroups;
+    L->buf_off[0] = off; off = align256(off + B * H * cap * R * esz);      // x_buf
+    L->buf_off[1] = off; off = align256(off + B * G * cap * C * esz);      // B_buf
+    L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // dt_buf
+  } else {
+    L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf
+    L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf
+    L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // g_buf
+    L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf
+    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf
+  }
+  *buf = off;
+  if (d->read_fmt == RSSM_READ_FP32) {
+    *rc = 0;
+  } else if (d->read_fmt == RSSM_READ_FP8_E4M3_ROW) {
+    L->rc_codes_off = 0;
+    L->rc_scales_off = align256(B * H * R * C);
+    *rc = align256(L->rc_scales_off + B * H * R * sizeof(float));
+  } else {
+    L->rc_codes_off = 0;
+    L->rc_scales_off = align256(B * H * R * C / 2);
+    *rc = align256(L->rc_scales_off + B * H * R * (C / 16));
+  }
+  off = 0;
+  L->meta_start_off = off; off = align256(off + B * 4);
+  L->meta_len_off = off; off = align256(off + B * 4);
+  L->meta_pending_off = off; off = align256(off + B * 4);
+  L->meta_flushes_off = off; off = align256(off + B * 4);
+  L->meta_arrivals_off = off; off = align256(off + B * 4);
+  L->meta_status_off = off; off = align256(off + 4);
+  *meta = off;
+}
+
+rssm::StepArgs step_args(const rssm_handle *h, int mode, int m) {
+  rssm::StepArgs a;
+  std::memset(&a, 0, sizeof a);
+  const rssm_layer_desc &d = h->d;
+  a.B = d.batch; a.H = d.nheads;
+  a.G = d.kind == RSSM_MAMBA2 ? d.ngroups : 1;
+  a.hpg = d.nheads / a.G;
+  a.R = d.headdim; a.C = d.dstate;
+  a.L = d.window; a.cap = (int)h->lay.cap;
+  a.m = m; a.mode = mode; a.auto_flush = d.auto_flush != 0;
+  a.out_scale = d.out_scale;
+  a.A = h->A; a.D = h->D;
+  a.hc = h->ckpt;
+  a.rc_codes = h->rc ? h->rc + h->lay.rc_codes_off : nullptr;
+  a.rc_scales = h->rc ? h->rc + h->lay.rc_scales_off : nullptr;
+  a.buf0 = h->buf + h->lay.buf_off[0];
+  a.buf1 = h->buf + h->lay.buf_off[1];
+  a.buf2 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[2]);
+  if (d.kind == RSSM_GDN) {
+    a.buf3 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[3]);
+    a.buf4 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[4]);
+  }
+  a.start = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_start_off);
+  a.len = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_len_off);
+  a.pending = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_pending_off);
+  a.flushes = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_flushes_off);
+  a.arrivals = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_arrivals_off);
+  a.status = reinterpret_cast<uint32_t *>(h->meta + h->lay.meta_status_off);
+  return a;
+}
+
+int n_inputs(const rssm_handle *h) { return h->d.kind == RSSM_MAMBA2 ? 4 : 5; }
+
+int check_inputs(const rssm_handle *h, const void *const *in, const void *out) {
+  if (!in) return fail(RSSM_ERR_INVALID_ARG, "in is NULL");
+  for (int i = 0; i < n_inputs(h); ++i) {
+    if (!in[i]) return fail(RSSM_ERR_INVALID_ARG, "in[%d] is NULL", i);
+    if (!aligned(in[i], 16)) return fail(RSSM_ERR_INVALID_ARG, "in[%d] is not 16-byte aligned", i);
+  }
+  if (!out) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
+  if (!aligned(out, 16)) return fail(RSSM_ERR_INVALID_ARG, "out is not 16-byte aligned");
+  if (h->d.kind == RSSM_MAMBA2 && (!h->A || !h->D))
+    return fail(RSSM_ERR_STATE, "Mamba-2 parameters not set (rssm_set_params)");
+  return RSSM_OK;
+}
+
+int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *out,
+                const int32_t *mask, cudaStream_t s) {
+  rssm::StepArgs a = step_args(h, mode, m);
+  if (in)
+    for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
+  a.out = static_cast<float *>(out);
+  a.mask = mask;
+  cudaError_t e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, s)
+                                           : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, s);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes, size_t *buf_bytes,
+                        size_t *read_copy_bytes, size_t *meta_bytes, rssm_layout *layout) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!ckpt_bytes || !buf_bytes || !read_copy_bytes || !meta_bytes)
+    return fail(RSSM_ERR_INVALID_ARG, "size outputs must not be NULL");
+  rssm_layout tmp;
+  compute_layout(desc, layout ? layout : &tmp, ckpt_bytes, buf_bytes, read_copy_bytes, meta_bytes);
+  return ok();
+}
+
+int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev, void *read_copy_dev,
+                void *meta_dev, rssm_handle **out) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!out) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!ckpt_dev || !buf_dev || !meta_dev)
+    return fail(RSSM_ERR_INVALID_ARG, "ckpt, buf and meta must not be NULL");
+  if (!aligned(ckpt_dev, 256) || !aligned(buf_dev, 256) || !aligned(meta_dev, 256))
+    return fail(RSSM_ERR_INVALID_ARG, "device buffers must be 256-byte aligned");
+  if (desc->read_fmt != RSSM_READ_FP32) {
+    if (!read_copy_dev) return fail(RSSM_ERR_INVALID_ARG, "read_fmt needs a read_copy buffer");
+    if (!aligned(read_copy_dev, 256)) return fail(RSSM_ERR_INVALID_ARG, "read_copy must be 256-byte aligned");
+  }
+  rssm_handle *h = new (std::nothrow) rssm_handle;
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "out of host memory");
+  std::memset(h, 0, sizeof *h);
+  h->d = *desc;
+  compute_layout(desc, &h->lay, &h->ckpt_bytes, &h->buf_bytes, &h->rc_bytes, &h->meta_bytes);
+  h->ckpt = static_cast<float *>(ckpt_dev);
+  h->buf = static_cast<uint8_t *>(buf_dev);
+  h->rc = desc->read_fmt == RSSM_READ_FP32 ? nullptr : static_cast<uint8_t *>(read_copy_dev);
+  h->meta = static_cast<uint8_t *>(meta_dev);
+  *out = h;
+  return ok();
+}
+
+int rssm_destroy(rssm_handle *h) {
+  delete h;
+  return ok();
+}
+
+int rssm_reset(rssm_handle *h, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  cudaError_t e = cudaMemsetAsync(h->meta, 0, h->meta_bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(meta)");
+  return ok();
+}
+
+int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.kind == RSSM_MAMBA2 && (!A_dev || !D_dev))
+    return fail(RSSM_ERR_INVALID_ARG, "A and D must not be NULL");
+  h->A = A_dev;
+  h->D = D_dev;
+  return ok();
+}
+
+int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  int rc = check_inputs(h, in, out_dev);
+  if (rc) return rc;
+  return launch_step(h, rssm::kDecode, 1, in, out_dev, nullptr, (cudaStream_t)stream);
+}
+
+int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.max_draft < 1) return fail(RSSM_ERR_STATE, "handle was created with max_draft = 0");
+  if (k < 1 || k > h->d.max_draft)
+    return fail(RSSM_ERR_CAPACITY, "k = %d outside [1, max_draft = %d]", k, h->d.max_draft);
+  int rc = check_inputs(h, in, out_dev);
+  if (rc) return rc;
+  return launch_step(h, rssm::kVerify, k, in, out_dev, nullptr, (cudaStream_t)stream);
+}
+
+int rssm_rollback(rssm_handle *h, const int32_t *n_reject_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!n_reject_dev) return fail(RSSM_ERR_INVALID_ARG, "n_reject is NULL");
+  rssm::StepArgs a = step_args(h, rssm::kVerify, 0);
+  cudaError_t e = rssm::rollback(a.B, n_reject_dev, a.len, a.pending, a.status, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "rollback launch");
+  return ok();
+}
+
+int rssm_flush(rssm_handle *h, const int32_t *row_mask_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.kind == RSSM_MAMBA2 && (!h->A || !h->D))
+    return fail(RSSM_ERR_STATE, "Mamba-2 parameters not set (rssm_set_params)");
+  return launch_step(h, rssm::kFlush, 0, nullptr, nullptr, row_mask_dev, (cudaStream_t)stream);
+}
+
+int rssm_quantize_read_copy(rssm_handle *h, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!h->rc) return fail(RSSM_ERR_STATE, "handle has no read copy (read_fmt = RSSM_READ_FP32)");
+  rssm::QuantArgs q;
+  q.rows = (size_t)h->d.batch * h->d.nheads * h->d.headdim;
+  q.C = h->d.dstate;
+  q.hc = h->ckpt;
+  q.codes = h->rc + h->lay.rc_codes_off;
+  q.scales = h->rc + h->lay.rc_scales_off;
+  cudaError_t e = rssm::quantize_read_copy(q, h->d.read_fmt, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
+}
+
+int rssm_conventional_step(rssm_handle *h, const float *state_in_dev, float *state_out_dev,
+                           const void *const *in, void *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!state_in_dev || !state_out_dev) return fail(RSSM_ERR_INVALID_ARG, "state pointers must not be NULL");
+  if (!aligned(state_in_dev, 16) || !aligned(state_out_dev, 16))
+    return fail(RSSM_ERR_INVALID_ARG, "state pointers must be 16-byte aligned");
+  int rc = check_inputs(h, in, out_dev);
+  if (rc) return rc;
+  rssm::ConvArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.B = h->d.batch; a.H = h->d.nheads;
+  a.G = h->d.kind == RSSM_MAMBA2 ? h->d.ngroups : 1;
+  a.hpg = a.H / a.G;
+  a.R = h->d.headdim; a.C = h->d.dstate;
+  a.out_scale = h->d.out_scale;
+  a.A = h->A; a.D = h->D;
+  a.state_in = state_in_dev; a.state_out = state_out_dev;
+  for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
+  a.out = static_cast<float *>(out_dev);
+  cudaError_t e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_conventional(a, h->d.in_dtype, (cudaStream_t)stream)
+                                           : rssm::gdn_conventional(a, h->d.in_dtype, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "conventional kernel launch");
+  return ok();
+}
+
+int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!out_dev) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
+  rssm::StepArgs a = step_args(h, rssm::kDecode, 0);
+  cudaError_t e = rssm::gather_bookkeeping(a.B, a.start, a.len, a.pending, a.flushes, out_dev,
+                                           (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "bookkeeping gather launch");
+  return ok();
+}
+
+int rssm_get_status(rssm_handle *h, uint32_t *bits, int clear, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!bits) return fail(RSSM_ERR_INVALID_ARG, "bits is NULL");
+  uint32_t *dev = reinterpret_cast<uint32_t *>(h->meta + h->lay.meta_status_off);
+  cudaError_t e = cudaMemcpyAsync(bits, dev, sizeof(uint32_t), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(dev, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  return ok();
+}
+
+const char *rssm_last_error_string(void) { return g_err.c_str(); }
+
+uint64_t rssm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

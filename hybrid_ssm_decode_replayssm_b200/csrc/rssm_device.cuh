@@ -1,0 +1,207 @@
+// Device helpers shared by the librssm kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "rssm_internal.h"
+
+namespace rssm {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------- loads
+// The checkpoint is streamed once per call: keep it out of L1 and mark it
+// evict-first in L2 so the window buffers (re-read every step) stay cached.
+__device__ __forceinline__ float4 ld_stream(const float *p) {
+  return __ldcs(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ void st_stream(float *p, float4 v) {
+  __stcs(reinterpret_cast<float4 *>(p), v);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// Copy `n` elements (n % 8 == 0, 16-byte aligned source) of type T from global
+// memory into fp32 shared memory, using the threads [t0, t0 + nt).
+template <typename T>
+__device__ __forceinline__ void stage_row(float *dst, const T *src, int n, int t, int nt) {
+  constexpr int kPer = 16 / sizeof(T);
+  for (int i = t; i < n / kPer; i += nt) {
+    uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+    const T *e = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) dst[i * kPer + c] = to_f32<T>(e[c]);
+  }
+}
+
+// Copy n elements of T (n % 8 == 0) global -> global (ring-buffer append).
+template <typename T>
+__device__ __forceinline__ void copy_row(T *dst, const T *src, int n, int t, int nt) {
+  constexpr int kPer = 16 / sizeof(T);
+  for (int i = t; i < n / kPer; i += nt)
+    reinterpret_cast<uint4 *>(dst)[i] = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+}
+
+// ------------------------------------------------------ warp reductions
+// Transposed reduction.  Each lane holds NV partial sums v[0..NV); lanes are
+// grouped in aligned groups of W consecutive lanes that must be summed.  At
+// every level the pair of lanes (lane, lane ^ O) trades half of its values so
+// the number of live values halves; once one value is left the remaining
+// levels are plain butterflies.  On return the lane's live values v[0..R),
+// R = max(1, NV / W), are complete sums of the original indices
+// tr_base<NV, W/2>(lane) + i.  NV and W are powers of two.
+template <int NV, int O>
+__device__ __forceinline__ void tr_sum(float *v, int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (NV > 1) {
+      constexpr int H = NV / 2;
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < H; ++i) {
+        const float keep = up ? v[i + H] : v[i];
+        const float send = up ? v[i] : v[i + H];
+        v[i] = keep + __shfl_xor_sync(kFull, send, O);
+      }
+      tr_sum<H, O / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(kFull, v[0], O);
+      tr_sum<1, O / 2>(v, lane);
+    }
+  }
+}
+
+template <int NV, int O>
+__device__ __forceinline__ int tr_base(int lane) {
+  if constexpr (O >= 1 && NV > 1) {
+    return ((lane & O) ? NV / 2 : 0) + tr_base<NV / 2, O / 2>(lane);
+  } else {
+    return 0;
+  }
+}
+
+// Max over aligned groups of W lanes (all lanes get the result).
+template <int W>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = W / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------- read-copy codecs
+// OCP E4M3 (satfinite, round to nearest even) and FP4 E2M1 via CUDA's
+// conversion functions; the divisions that feed them are IEEE fp32 divisions.
+__device__ __forceinline__ uint32_t enc_e4m3(float x) {
+  return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float dec_e4m3(uint32_t c) {
+  __half_raw r = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+  return __half2float(__half(r));
+}
+__device__ __forceinline__ uint32_t enc_e2m1(float x) {
+  return (uint32_t)__nv_cvt_float_to_fp4(x, __NV_E2M1, cudaRoundNearest) & 0xFu;
+}
+__device__ __forceinline__ float dec_e2m1(uint32_t c) {
+  __half_raw r = __nv_cvt_fp4_to_halfraw((__nv_fp4_storage_t)c, __NV_E2M1);
+  return __half2float(__half(r));
+}
+// Four E4M3 codes packed little-endian in w -> fp32.
+__device__ __forceinline__ void dec_e4m3x4(uint32_t w, float s, float4 &o) {
+  __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+  o = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
+}
+// Four E2M1 codes packed in 16 bits (element 0 in the lowest nibble) -> fp32.
+__device__ __forceinline__ void dec_e2m1x4(uint32_t w, float s, float4 &o) {
+  __half2_raw lo = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(w & 0xFFu), __NV_E2M1);
+  __half2_raw hi = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w >> 8) & 0xFFu), __NV_E2M1);
+  float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+  o = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
+}
+
+__device__ __forceinline__ float f4get(const float4 &v, int c) {
+  return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+}
+
+// Quantise the 4 elements a lane holds of one state row (columns c0..c0+3) into
+// the read copy, and return the dequantised values the reads will see.
+//   FP8 row:  lanes of the row (a group of LPR lanes) share one fp32 scale.
+//   NVFP4:    groups of 4 lanes (16 elements) share one E4M3 scale.
+template <int RF, int LPR>
+__device__ __forceinline__ float4 quantize4(const float4 v, uint8_t *codes_row, void *scales,
+                                            size_t row, int ncols, int c0, int lane) {
+  float4 out;
+  if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+    float am = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    am = group_max<LPR>(am);
+    const float s = am / 448.0f;
+    uint32_t w = 0;
+    if (s != 0.0f) {
+      w = enc_e4m3(v.x / s) | (enc_e4m3(v.y / s) << 8) | (enc_e4m3(v.z / s) << 16) |
+          (enc_e4m3(v.w / s) << 24);
+    }
+    *reinterpret_cast<uint32_t *>(codes_row + c0) = w;
+    if ((lane % LPR) == 0) reinterpret_cast<float *>(scales)[row] = s;
+    dec_e4m3x4(w, s, out);
+  } else {
+    float am = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    am = group_max<4>(am);
+    const uint32_t sc = enc_e4m3(am / 6.0f);
+    const float sv = dec_e4m3(sc);
+    uint32_t w = 0;
+    if (sv != 0.0f) {
+      w = enc_e2m1(v.x / sv) | (enc_e2m1(v.y / sv) << 4) | (enc_e2m1(v.z / sv) << 8) |
+          (enc_e2m1(v.w / sv) << 12);
+    }
+    *reinterpret_cast<uint16_t *>(codes_row + c0 / 2) = (uint16_t)w;
+    if ((c0 % 16) == 0)
+      reinterpret_cast<uint8_t *>(scales)[row * (ncols / 16) + c0 / 16] = (uint8_t)sc;
+    dec_e2m1x4(w, sv, out);
+  }
+  return out;
+}
+
+// Load the 4 read-copy elements of (row, c0..c0+3) and dequantise them.
+template <int RF>
+__device__ __forceinline__ float4 load_read_copy4(const uint8_t *codes_row, const void *scales,
+                                                  size_t row, int ncols, int c0) {
+  float4 out;
+  if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+    const uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(codes_row + c0));
+    const float s = __ldg(reinterpret_cast<const float *>(scales) + row);
+    dec_e4m3x4(w, s, out);
+  } else {
+    const uint32_t w = __ldcs(reinterpret_cast<const unsigned short *>(codes_row + c0 / 2));
+    const uint32_t sc = __ldg(reinterpret_cast<const uint8_t *>(scales) + row * (ncols / 16) + c0 / 16);
+    dec_e2m1x4(w, dec_e4m3(sc), out);
+  }
+  return out;
+}
+
+// Arrival counter: returns true in exactly one thread (thread 0 of the last of
+// `expected` CTAs to arrive for this counter).  Call after __syncthreads().
+__device__ __forceinline__ bool last_arrival(int32_t *counter, int expected) {
+  bool last = false;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(counter, 1) == expected - 1;
+    if (last) *counter = 0;
+  }
+  return last;
+}
+
+}  // namespace rssm

@@ -1,0 +1,79 @@
+// Internal interface between the C-ABI host code and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/rssm.h"
+
+namespace rssm {
+
+enum StepMode { kDecode = 0, kVerify = 1, kFlush = 2 };
+
+constexpr int kMaxWindow = 32;
+constexpr int kMaxDraft = 8;
+
+// Everything a replay kernel needs about one call.  Pointers are device
+// pointers into the caller's buffers.
+struct StepArgs {
+  // shape
+  int B, H, G, hpg;      // hpg = heads per group (Mamba-2)
+  int R, C;              // state rows / columns (P, N  or  dv, dk)
+  int L, cap;            // window and ring capacity
+  int m;                 // tokens appended by this call (1 decode, k verify, 0 flush)
+  int mode;              // StepMode
+  int auto_flush;
+  float out_scale;       // GDN
+  // parameters (Mamba-2)
+  const float *A, *D;
+  // checkpoint and read copy
+  float *hc;
+  uint8_t *rc_codes;
+  void *rc_scales;
+  // ring buffers (layer specific, see rssm.h)
+  void *buf0, *buf1;     // Mamba-2: x_buf, B_buf     GDN: k_buf, v_buf
+  float *buf2, *buf3, *buf4;  // Mamba-2: dt_buf     GDN: g_buf, beta_buf, w_buf
+  // per-call inputs / outputs
+  const void *in[5];
+  float *out;
+  const int32_t *mask;   // flush row mask (nullable)
+  // bookkeeping
+  int32_t *start, *len, *pending, *flushes, *arrivals;
+  uint32_t *status;
+};
+
+struct ConvArgs {
+  int B, H, G, hpg, R, C;
+  float out_scale;
+  const float *A, *D;
+  const float *state_in;
+  float *state_out;
+  const void *in[5];
+  float *out;
+};
+
+struct QuantArgs {
+  size_t rows;           // B*H*R
+  int C;
+  const float *hc;
+  uint8_t *codes;
+  void *scales;
+};
+
+// Launchers return cudaGetLastError() of their launch.
+cudaError_t mamba2_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
+cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s);
+cudaError_t gdn_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
+cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s);
+cudaError_t quantize_read_copy(const QuantArgs &a, int read_fmt, cudaStream_t s);
+cudaError_t rollback(int B, const int32_t *n_reject, int32_t *len, int32_t *pending,
+                     uint32_t *status, cudaStream_t s);
+cudaError_t gather_bookkeeping(int B, const int32_t *start, const int32_t *len,
+                               const int32_t *pending, const int32_t *flushes, int32_t *out,
+                               cudaStream_t s);
+
+bool mamba2_supported(int R, int C);
+bool gdn_supported(int R, int C);
+
+}  // namespace rssm

@@ -1,0 +1,132 @@
+"""The C-ABI library loads, exports every function include/rssm.h declares, and
+its host-side checks behave as documented (no GPU and no device memory used)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from hybrid_ssm_decode_replayssm_b200 import rssm
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "rssm.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z0-9_]+\s*\*?\s*(rssm_[a-z0-9_]+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(rssm.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = rssm.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def _desc(**kw):
+    base = dict(kind=rssm.RSSM_MAMBA2, batch=4, nheads=8, headdim=64, dstate=128, ngroups=2,
+                window=16, max_draft=4, in_dtype=rssm.RSSM_BF16, read_fmt=rssm.RSSM_READ_FP32)
+    base.update(kw)
+    return rssm.make_desc(**base)
+
+
+def _sizes(desc):
+    s = [C.c_size_t() for _ in range(4)]
+    lay = rssm.Layout()
+    code = rssm.lib().rssm_workspace_size(C.byref(desc), *[C.byref(x) for x in s], C.byref(lay))
+    return code, [x.value for x in s], lay
+
+
+def test_workspace_layout_mamba2():
+    code, (ck, buf, rc, meta), lay = _sizes(_desc())
+    assert code == rssm.RSSM_OK
+    B, H, P, N, G, cap = 4, 8, 64, 128, 2, 20
+    assert lay.cap == cap and ck == B * H * P * N * 4 and rc == 0
+    assert lay.buf_off[0] == 0
+    assert lay.buf_off[1] >= B * H * cap * P * 2 and lay.buf_off[1] % 256 == 0
+    assert lay.buf_off[2] >= lay.buf_off[1] + B * G * cap * N * 2
+    assert buf >= lay.buf_off[2] + B * H * cap * 4
+    assert meta >= lay.meta_status_off + 4
+
+
+@pytest.mark.parametrize("fmt", [rssm.RSSM_READ_FP8_E4M3_ROW, rssm.RSSM_READ_NVFP4])
+def test_workspace_layout_read_copy(fmt):
+    code, (ck, buf, rc, meta), lay = _sizes(_desc(read_fmt=fmt))
+    assert code == rssm.RSSM_OK
+    rows, n = 4 * 8 * 64, 128
+    if fmt == rssm.RSSM_READ_FP8_E4M3_ROW:
+        codes_bytes, scale_bytes = rows * n, rows * 4            # 1 byte/elem, fp32 per row
+    else:
+        codes_bytes, scale_bytes = rows * n // 2, rows * n // 16  # 4 bits/elem, e4m3 per 16
+    assert lay.rc_codes_off == 0 and lay.rc_scales_off >= codes_bytes
+    assert lay.rc_scales_off % 256 == 0 and rc >= lay.rc_scales_off + scale_bytes
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kind=7), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(batch=0), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(ngroups=3), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(window=0), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(window=33), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(max_draft=9), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(window=2, max_draft=3), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(in_dtype=5), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(read_fmt=9), rssm.RSSM_ERR_INVALID_ARG),
+    (dict(headdim=48), rssm.RSSM_ERR_UNSUPPORTED),
+    (dict(dstate=96), rssm.RSSM_ERR_UNSUPPORTED),
+])
+def test_descriptor_validation(kw, code):
+    got, _, _ = _sizes(_desc(**kw))
+    assert got == code
+    assert rssm.lib().rssm_last_error_string()
+
+
+def test_create_checks_pointers_and_enqueues_nothing():
+    L = rssm.lib()
+    d = _desc()
+    h = C.c_void_p()
+    fake = 1 << 20                                          # never dereferenced by rssm_create
+    assert L.rssm_create(C.byref(d), None, fake, None, fake, C.byref(h)) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_create(C.byref(d), fake + 16, fake, None, fake, C.byref(h)) == rssm.RSSM_ERR_INVALID_ARG
+    d2 = _desc(read_fmt=rssm.RSSM_READ_NVFP4)
+    assert L.rssm_create(C.byref(d2), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_create(C.byref(d), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        ins = (C.c_void_p * 4)(fake, fake, fake, fake)
+        # parameters not set -> STATE, before anything is launched
+        assert L.rssm_decode_step(h, ins, fake, None) == rssm.RSSM_ERR_STATE
+        assert L.rssm_set_params(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_set_params(h, fake, fake) == rssm.RSSM_OK
+        bad = (C.c_void_p * 4)(fake, None, fake, fake)
+        assert L.rssm_decode_step(h, bad, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+        mis = (C.c_void_p * 4)(fake, fake + 2, fake, fake)
+        assert L.rssm_decode_step(h, mis, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_decode_step(h, ins, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_verify(h, 0, ins, fake, None) == rssm.RSSM_ERR_CAPACITY
+        assert L.rssm_verify(h, 5, ins, fake, None) == rssm.RSSM_ERR_CAPACITY
+        assert L.rssm_rollback(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_quantize_read_copy(h, None) == rssm.RSSM_ERR_STATE
+        assert L.rssm_conventional_step(h, None, fake, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_get_bookkeeping(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_get_status(h, None, 0, None) == rssm.RSSM_ERR_INVALID_ARG
+    finally:
+        assert L.rssm_destroy(h) == rssm.RSSM_OK
+    d0 = _desc(max_draft=0)
+    assert L.rssm_create(C.byref(d0), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    L.rssm_set_params(h, fake, fake)
+    assert L.rssm_verify(h, 1, ins, fake, None) == rssm.RSSM_ERR_STATE
+    L.rssm_destroy(h)
+
+
+def test_null_handle_everywhere():
+    L = rssm.lib()
+    for name in ["rssm_reset", "rssm_quantize_read_copy"]:
+        assert getattr(L, name)(None, None) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_flush(None, None, None) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_decode_step(None, None, None, None) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_launch_count() >= 0
