@@ -11,12 +11,10 @@
 // folded in when it fills; drafts are appended and rolled back by pointer; a
 // low-precision copy of the checkpoint may serve the reads.
 //
-// One CTA owns one (sequence b, head h): its checkpoint tile [P, N] fp32 is
-// streamed from HBM into registers with 128-bit loads (8 warps; a warp covers
-// P/8 rows, a lane 4 consecutive columns of a row), the window's x / B / dt and
-// the new tokens' C are staged in shared memory, and row dot products use a
-// transposed warp reduction.  The tile is written back only when the row is
-// folded (window full, or the new tokens would not fit).
+// The replay kernel streams each head's checkpoint tile (or its read copy)
+// through shared memory with 1-D TMA bulk copies, several heads in flight per
+// CTA; see m2_replay_kernel.  The conventional kernel keeps one CTA per
+// (sequence, head) and holds the tile in registers.
 #include <algorithm>
 
 #include "rssm_device.cuh"
@@ -27,35 +25,91 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
-template <int P, int N>
+// Tile mapping: W warps cover the P rows of a [P, N] fp32 tile; a lane holds 4
+// consecutive columns of a row (float4), LPR lanes cover one row, a warp
+// instruction covers RPI rows.
+template <int P, int N, int W = kWarps>
 struct Tile {
   static constexpr int LPR = N / 4;     // lanes per state row
   static constexpr int RPI = 32 / LPR;  // rows covered by one warp instruction
-  static constexpr int RPW = P / kWarps;
+  static constexpr int RPW = P / W;     // rows per warp
   static constexpr int NLD = RPW / RPI; // float4 per lane
   static_assert(N == 64 || N == 128, "dstate 64 or 128");
   static_assert(RPW % RPI == 0, "headdim must cover whole warp instructions");
 };
 
+template <int RF, int P, int N>
+constexpr int tile_bytes() {
+  return RF == RSSM_READ_FP32 ? P * N * 4 : RF == RSSM_READ_FP8_E4M3_ROW ? P * N : P * N / 2;
+}
+template <int RF, int P, int N>
+constexpr int scale_bytes() {
+  return RF == RSSM_READ_FP32 ? 0 : RF == RSSM_READ_FP8_E4M3_ROW ? P * 4 : P * (N / 16);
+}
 template <int RF, int N>
 constexpr int rc_row_bytes() { return RF == RSSM_READ_NVFP4 ? N / 2 : N; }
 
-// t <- dec * t + sum_{i0 <= i < i1} fw[i] x_i[row] B_i[cols]   (rank-(i1-i0) fold)
-template <int P, int N>
-__device__ __forceinline__ void fold_tile(float4 (&t)[Tile<P, N>::NLD], const float *s_fw, float dec,
-                                          int i0, int i1, const float *s_x, const float *s_B,
+// Suffix sums over a warp: lanes l < len hold v (the others 0).  Returns in
+// `after` the sum of v over lanes l' > l (direct sums of the terms, no
+// differences of prefix sums) and in `total` the sum over all lanes.
+__device__ __forceinline__ void suffix_scan(float v, int lane, float &after, float &total) {
+  float incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float t = __shfl_down_sync(kFull, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  after = __shfl_down_sync(kFull, incl, 1);
+  if (lane == 31) after = 0.0f;
+  total = __shfl_sync(kFull, incl, 0);
+}
+
+// Stage layout for one head: [read tile | scales | committed x rows (L) | new x rows (MAXM)].
+struct Stage {
+  uint8_t *base;
+  int xoff, xrow, n, L;
+  template <typename Tin>
+  __device__ __forceinline__ const Tin *row(int i) const {  // x row of window entry i
+    const int r = i < n ? i : L + (i - n);
+    return reinterpret_cast<const Tin *>(base + xoff + (size_t)r * xrow);
+  }
+  template <typename Tin>
+  __device__ __forceinline__ float x(int i, int p) const { return to_f32<Tin>(row<Tin>(i)[p]); }
+  // x_i at rows p0, p0 + step, ..., K values (one vector load when step == 1).
+  template <typename Tin, int K>
+  __device__ __forceinline__ void xs(int i, int p0, int step, float (&o)[K]) const {
+    const Tin *r = row<Tin>(i) + p0;
+    if (step == 1 && (K * sizeof(Tin)) % 16 == 0) {
+#pragma unroll
+      for (int c = 0; c < (int)(K * sizeof(Tin) / 16); ++c) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(r + c * (16 / sizeof(Tin)));
+        const Tin *e = reinterpret_cast<const Tin *>(&raw);
+#pragma unroll
+        for (int q = 0; q < (int)(16 / sizeof(Tin)); ++q) o[c * (16 / sizeof(Tin)) + q] = to_f32<Tin>(e[q]);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < K; ++q) o[q] = to_f32<Tin>(r[q * step]);
+    }
+  }
+};
+
+// t <- dec * t + sum_{i0 <= i < i1} fw[i - i0] x_i[row] B_i[cols]   (rank-(i1-i0) fold)
+template <int P, int N, int W, typename Tin>
+__device__ __forceinline__ void fold_tile(float4 (&t)[Tile<P, N, W>::NLD], const float *s_fw, float dec,
+                                          int i0, int i1, const Stage &stg, const float *s_B,
                                           int row0, int c0) {
-  using T = Tile<P, N>;
+  using T = Tile<P, N, W>;
 #pragma unroll
   for (int l = 0; l < T::NLD; ++l) {
     t[l].x *= dec; t[l].y *= dec; t[l].z *= dec; t[l].w *= dec;
   }
   for (int i = i0; i < i1; ++i) {
     const float4 bv = *reinterpret_cast<const float4 *>(s_B + i * N + c0);
-    const float fw = s_fw[i];
+    const float fw = s_fw[i - i0];
 #pragma unroll
     for (int l = 0; l < T::NLD; ++l) {
-      const float xr = fw * s_x[i * P + row0 + l * T::RPI];
+      const float xr = fw * stg.x<Tin>(i, row0 + l * T::RPI);
       t[l].x = fmaf(xr, bv.x, t[l].x);
       t[l].y = fmaf(xr, bv.y, t[l].y);
       t[l].z = fmaf(xr, bv.z, t[l].z);
@@ -64,285 +118,447 @@ __device__ __forceinline__ void fold_tile(float4 (&t)[Tile<P, N>::NLD], const fl
   }
 }
 
-// Outputs y_j for the m new tokens from the read view `v` (registers).
-template <int P, int N, int MAXM>
-__device__ __forceinline__ void outputs(const float4 (&v)[Tile<P, N>::NLD], const StepArgs &a,
-                                        const float *s_C, const float *s_x, const float *s_coef,
-                                        const float *s_dec, int b, int h, int n, int w0,
-                                        int warp, int lane, int c0) {
-  using T = Tile<P, N>;
+// Outputs of the m new tokens from the read view v (registers).  Lane l of a
+// row's lane group adds the window terms of entries i = w0 + l (+ LPR, ...)
+// to its partial sums, so that one transposed reduction over the row's lanes
+// yields  dec_j (v . C_j) + sum_i coef_ji x_i[row]  for every row and output;
+// the lanes left holding copies of a sum let one of them add D x_e and store.
+template <int P, int N, int W, typename Tin, int MAXM>
+__device__ __forceinline__ void outputs(const float4 (&v)[Tile<P, N, W>::NLD], const StepArgs &a,
+                                        const float *s_C, const float *hcoef, const float *hdec,
+                                        const Stage &stg, int b, int h, int n, int w0, int row0,
+                                        int lane, int c0) {
+  using T = Tile<P, N, W>;
   constexpr int NV = T::NLD * MAXM;
+  constexpr int DUP = NV >= T::LPR ? 1 : T::LPR / NV;
   float part[NV];
 #pragma unroll
   for (int j = 0; j < MAXM; ++j) {
     const float4 cv = *reinterpret_cast<const float4 *>(s_C + j * N + c0);
+    const float dj = hdec[j];
 #pragma unroll
     for (int l = 0; l < T::NLD; ++l)
-      part[l * MAXM + j] = v[l].x * cv.x + v[l].y * cv.y + v[l].z * cv.z + v[l].w * cv.w;
+      part[l * MAXM + j] = dj * (v[l].x * cv.x + v[l].y * cv.y + v[l].z * cv.z + v[l].w * cv.w);
+  }
+  const int emax = n + a.m - 1;   // last entry of the output window
+  for (int i = w0 + lane % T::LPR; i <= emax; i += T::LPR) {
+    float xr[T::NLD];
+    stg.xs<Tin, T::NLD>(i, row0, T::RPI, xr);
+#pragma unroll
+    for (int j = 0; j < MAXM; ++j) {
+      const float cj = hcoef[j * 32 + (i - w0)];   // 0 for entries after e_j
+#pragma unroll
+      for (int l = 0; l < T::NLD; ++l) part[l * MAXM + j] = fmaf(cj, xr[l], part[l * MAXM + j]);
+    }
   }
   tr_sum<NV, T::LPR / 2>(part, lane);
   const int base = tr_base<NV, T::LPR / 2>(lane);
   constexpr int R = NV >= T::LPR ? NV / T::LPR : 1;
-  const bool writer = NV >= T::LPR || (lane & (T::LPR / NV - 1)) == 0;
+  const bool writer = (lane & (DUP - 1)) == 0;
   const float Dh = __ldg(a.D + h);
-  const int cap = a.cap;
 #pragma unroll
-  for (int q = 0; q < R; ++q) {
-    const int idx = base + q, l = idx / MAXM, j = idx % MAXM;
+  for (int r = 0; r < R; ++r) {
+    const int idx = base + r, l = idx / MAXM, j = idx % MAXM;
+    const int row = row0 + l * T::RPI;   // lanes keep their row group through the reduction
     if (writer && j < a.m) {
-      const int row = warp * T::RPW + l * T::RPI + lane / T::LPR;
       const int e = n + j;
-      float y = s_dec[j] * part[q];
-      for (int i = w0; i <= e; ++i) y = fmaf(s_coef[j * cap + i], s_x[i * P + row], y);
-      y = fmaf(Dh, s_x[e * P + row], y);
-      a.out[(((size_t)b * a.m + j) * a.H + h) * P + row] = y;
+      a.out[(((size_t)b * a.m + j) * a.H + h) * P + row] = fmaf(Dh, stg.x<Tin>(e, row), part[r]);
     }
   }
 }
 
+// Row decision shared by the producer and the consumers of a replay CTA (both
+// read the same pointers, so they take the same branch).
+struct RowPlan {
+  int st, n;
+  bool refuse, pre, post;
+  unsigned bit;
+};
+__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
+  RowPlan r;
+  r.st = a.start[b];
+  r.n = a.len[b];
+  const int pend = a.pending[b];
+  r.refuse = r.pre = r.post = false;
+  r.bit = 0;
+  if (a.mode == kFlush) {
+    if (a.mask != nullptr && a.mask[b] == 0) r.refuse = true;
+    else if (pend != 0) { r.refuse = true; r.bit = RSSM_STATUS_STATE; }
+    else if (r.n == 0) r.refuse = true;
+    else r.pre = true;
+  } else if (pend != 0) {
+    r.refuse = true;
+    r.bit = RSSM_STATUS_STATE;
+  } else {
+    r.pre = r.n + a.m > a.L;
+    if (r.pre && !a.auto_flush) {
+      r.refuse = true;
+      r.bit = RSSM_STATUS_CAPACITY;
+    }
+    r.post = !r.refuse && a.mode == kDecode && a.auto_flush && ((r.pre ? 0 : r.n) + 1 == a.L);
+  }
+  return r;
+}
+
+constexpr int kGroupWarps = 8;                  // consumer warps sharing one head
+constexpr int kGroups = 2;                      // consumer groups, alternating items
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kConsumers = kGroups * kGroupThreads;
+constexpr int kReplayThreads = kConsumers + 32; // + one producer warp
+constexpr int kMaxStages = 16;
+
+// The replay kernel: persistent and warp-specialised.  CTA c works through the
+// items c, c + grid, ... where an item is one (sequence b, group g, chunk of
+// `hc` heads); its heads are numbered in one sequence across the CTA's items
+// (seq = k * hc + jh), stage = seq % stages, use u = seq / stages.
+//  * Producer warp (one lane): for each head in sequence, waits until the
+//    consumers have released its stage (empty barrier, phase u - 1), then
+//    requests with 1-D TMA bulk copies the head's read tile (fp32, or FP8/NVFP4
+//    codes and scales), its committed window rows of x and the new tokens' x
+//    rows, all completing on the stage's full barrier.  It reads each item's
+//    ring pointers itself, ahead of the consumers.
+//  * Two consumer groups of 8 warps take alternate items, so that one group's
+//    item prologue (pointers, B window, C rows, B.C products, dt windows, every
+//    head's window scalars) overlaps the other group's heads.  Per head, each
+//    warp of the group takes P/8 rows: optional pre-fold, outputs (window
+//    terms merged into the row reductions), optional window-full fold; then it
+//    releases the stage.  There is no block-wide barrier after the start.
 template <int P, int N, typename Tin, int RF, int MAXM>
-__global__ void __launch_bounds__(kThreads) m2_step_kernel(const StepArgs a) {
-  using T = Tile<P, N>;
-  extern __shared__ float4 smem4[];
-  float *smem = reinterpret_cast<float *>(smem4);
-  const int cap = a.cap;
-  float *s_x = smem;                     // [cap][P]   window x (fp32)
-  float *s_B = s_x + cap * P;            // [cap][N]   window B
-  float *s_C = s_B + cap * N;            // [MAXM][N]  new tokens' C
-  float *s_dt = s_C + MAXM * N;          // [cap]
-  float *s_a = s_dt + cap;               // [cap]      dt * A
-  float *s_bc = s_a + cap;               // [MAXM][cap] B_i . C_j
-  float *s_coef = s_bc + MAXM * cap;     // [MAXM][cap] window coefficients
-  float *s_fwpre = s_coef + MAXM * cap;  // [cap]      fold weights (pre-fold)
-  float *s_fwpost = s_fwpre + cap;       // [cap]      fold weights (window-full fold)
-  float *s_dec = s_fwpost + cap;         // [MAXM + 2] decays: outputs, pre, post
-  __shared__ int s_book[3];
+__global__ void __launch_bounds__(kReplayThreads, 1)
+    m2_replay_kernel(const StepArgs a, const int hc, const int stages) {
+  using T = Tile<P, N, kGroupWarps>;
+  constexpr int XROW = P * (int)sizeof(Tin);
+  constexpr int TB = tile_bytes<RF, P, N>();
+  constexpr int SB = scale_bytes<RF, P, N>();
+  constexpr int RB = rc_row_bytes<RF, N>();
+  constexpr int HS = MAXM * 32 + MAXM + 64 + 2;   // per-head scalars
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
+  // stage_use[s] = the use index u the producer last requested on stage s.  A
+  // parity wait is exact only when the waiter is at most one phase ahead of
+  // the barrier; a consumer group that skips the other group's item could be
+  // further ahead, so it first waits for stage_use[s] == u.
+  __shared__ int stage_use[kMaxStages];
+  __shared__ int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x / a.H, h = blockIdx.x - b * a.H, g = h / a.hpg;
+  const int L = a.L, cap = a.cap, m = a.m, WMAX = L + MAXM;
+  const int nchunk = a.hpg / hc;
+  const int nitems = a.B * a.G * nchunk;
+  const int my_items = (int)blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int total_seq = my_items * hc;
+  const int XOFF = TB + SB;
+  const size_t stage_bytes = ((size_t)XOFF + (size_t)(L + MAXM) * XROW + 127) & ~(size_t)127;
+  // each group's region starts on a 128-byte boundary (float4 reads of B and C rows)
+  const int group_floats = (WMAX * N + MAXM * N + hc * WMAX + MAXM * WMAX + hc * HS + 31) & ~31;
+
+  const Tin *xin = reinterpret_cast<const Tin *>(a.in[0]);
+  const Tin *Bin = reinterpret_cast<const Tin *>(a.in[1]);
+  const Tin *Cin = reinterpret_cast<const Tin *>(a.in[2]);
+  const Tin *dtin = reinterpret_cast<const Tin *>(a.in[3]);
+  Tin *xring = reinterpret_cast<Tin *>(a.buf0);
+  volatile int *abort = &abort_flag;
+
   if (tid == 0) {
-    s_book[0] = a.start[b];
-    s_book[1] = a.len[b];
-    s_book[2] = a.pending[b];
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGroupWarps);
+      stage_use[s] = -1;
+    }
+    abort_flag = 0;
+    mbar_fence_init();
   }
   __syncthreads();
-  const int st = s_book[0], n = s_book[1], pend = s_book[2], m = a.m;
 
-  // Row decisions; every CTA of sequence b takes the same ones.
-  bool pre, post = false;
-  if (a.mode == kFlush) {
-    if (a.mask != nullptr && a.mask[b] == 0) return;
-    if (pend != 0) {
-      if (h == 0 && tid == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_STATE);
-      return;
-    }
-    if (n == 0) return;
-    pre = true;
-  } else {
-    if (pend != 0) {
-      if (h == 0 && tid == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_STATE);
-      return;
-    }
-    pre = n + m > a.L;
-    if (pre && !a.auto_flush) {
-      if (h == 0 && tid == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_CAPACITY);
-      return;
-    }
-    post = a.mode == kDecode && a.auto_flush && ((pre ? 0 : n) + 1 == a.L);
-  }
-  const int w0 = pre ? n : 0;  // first entry of the output window
-  const int ntot = n + m;
-  const bool need_f32 = (RF == RSSM_READ_FP32) || pre || post;
+  auto item_of = [&](int k, int &b, int &g, int &chunk) {
+    const int item = (int)blockIdx.x + k * (int)gridDim.x;
+    b = item / (a.G * nchunk);
+    const int rem = item - b * a.G * nchunk;
+    g = rem / nchunk;
+    chunk = rem - g * nchunk;
+  };
 
-  const size_t bh = (size_t)b * a.H + h;
-  float *hc = a.hc + bh * P * N;
-  const int row0 = warp * T::RPW + lane / T::LPR;
-  const int c0 = (lane % T::LPR) * 4;
-  constexpr int RB = rc_row_bytes<RF, N>();
-  uint8_t *rc = (RF != RSSM_READ_FP32) ? a.rc_codes + bh * P * RB : nullptr;
-
-  // 1. Stream the checkpoint tile (and/or its read copy) into registers.
-  float4 st4[T::NLD];
-  float4 view[T::NLD];
-  if (need_f32) {
-#pragma unroll
-    for (int l = 0; l < T::NLD; ++l) st4[l] = ld_stream(hc + (size_t)(row0 + l * T::RPI) * N + c0);
-  }
-  if constexpr (RF != RSSM_READ_FP32) {
-    if (!pre && m > 0) {
-#pragma unroll
-      for (int l = 0; l < T::NLD; ++l) {
-        const int row = row0 + l * T::RPI;
-        view[l] = load_read_copy4<RF>(rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0);
+  if (warp == kConsumers / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    int cur_k = -1, b = 0, g = 0, chunk = 0, jh = 0, s = 0, u = 0;
+    RowPlan rp{};
+    int issued = 0;
+    for (int seq = 0; seq < total_seq; ++seq) {
+      if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
+        atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
+        break;
       }
-    }
-  }
-
-  // 2. Stage the window (committed entries, then the new tokens) in shared
-  //    memory and append the new tokens to the ring.
-  constexpr int kPer = 16 / sizeof(Tin);
-  constexpr int XV = P / kPer, BV = N / kPer;
-  const Tin *xbuf = reinterpret_cast<const Tin *>(a.buf0) + bh * cap * P;
-  const Tin *Bbuf = reinterpret_cast<const Tin *>(a.buf1) + ((size_t)b * a.G + g) * cap * N;
-  for (int idx = tid; idx < n * (XV + BV); idx += kThreads) {
-    const int i = idx / (XV + BV), r = idx - i * (XV + BV);
-    const int slot = (st + i) % cap;
-    const Tin *src = r < XV ? xbuf + slot * P + r * kPer : Bbuf + slot * N + (r - XV) * kPer;
-    float *dst = r < XV ? s_x + i * P + r * kPer : s_B + i * N + (r - XV) * kPer;
-    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src));
-    const Tin *e = reinterpret_cast<const Tin *>(&raw);
-#pragma unroll
-    for (int c = 0; c < kPer; ++c) dst[c] = to_f32<Tin>(e[c]);
-  }
-  for (int i = tid; i < n; i += kThreads) s_dt[i] = a.buf2[bh * cap + (st + i) % cap];
-  {
-    const Tin *xin = reinterpret_cast<const Tin *>(a.in[0]);
-    const Tin *Bin = reinterpret_cast<const Tin *>(a.in[1]);
-    const Tin *Cin = reinterpret_cast<const Tin *>(a.in[2]);
-    const Tin *dtin = reinterpret_cast<const Tin *>(a.in[3]);
-    Tin *xring = reinterpret_cast<Tin *>(a.buf0) + bh * cap * P;
-    Tin *Bring = reinterpret_cast<Tin *>(a.buf1) + ((size_t)b * a.G + g) * cap * N;
-    const bool group_writer = (h % a.hpg) == 0;
-    for (int idx = tid; idx < m * (XV + 2 * BV); idx += kThreads) {
-      const int j = idx / (XV + 2 * BV), r = idx - j * (XV + 2 * BV);
-      const int slot = (st + n + j) % cap;   // same slot with or without a pre-fold
-      const size_t tok = (size_t)b * m + j;
-      const Tin *src;
-      float *dst;
-      Tin *ring = nullptr;
-      if (r < XV) {
-        src = xin + (tok * a.H + h) * P + r * kPer;
-        dst = s_x + (n + j) * P + r * kPer;
-        ring = xring + slot * P + r * kPer;
-      } else if (r < XV + BV) {
-        src = Bin + (tok * a.G + g) * N + (r - XV) * kPer;
-        dst = s_B + (n + j) * N + (r - XV) * kPer;
-        if (group_writer) ring = Bring + slot * N + (r - XV) * kPer;
+      if (cur_k < 0 || jh == hc) {
+        ++cur_k;
+        jh = 0;
+        item_of(cur_k, b, g, chunk);
+        rp = plan_row(a, b);
+      }
+      issued = seq + 1;
+      if (rp.refuse) {
+        mbar_arrive(&full[s]);
       } else {
-        src = Cin + (tok * a.G + g) * N + (r - XV - BV) * kPer;
-        dst = s_C + j * N + (r - XV - BV) * kPer;
+        const int h = g * a.hpg + chunk * hc + jh;
+        const size_t bh = (size_t)b * a.H + h;
+        uint8_t *dst = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + (m + rp.n) * XROW));
+        if constexpr (RF == RSSM_READ_FP32) {
+          bulk_g2s(dst, a.hc + bh * P * N, TB, &full[s]);
+        } else {
+          bulk_g2s(dst, a.rc_codes + bh * TB, TB, &full[s]);
+          bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + bh * SB, SB, &full[s]);
+        }
+        if (rp.n > 0) {
+          const Tin *src = xring + bh * cap * P;
+          const int c1 = rp.n < cap - rp.st ? rp.n : cap - rp.st;
+          bulk_g2s(dst + XOFF, src + (size_t)rp.st * P, c1 * XROW, &full[s]);
+          if (rp.n > c1) bulk_g2s(dst + XOFF + c1 * XROW, src, (rp.n - c1) * XROW, &full[s]);
+        }
+        for (int j = 0; j < m; ++j)
+          bulk_g2s(dst + XOFF + (L + j) * XROW, xin + (((size_t)b * m + j) * a.H + h) * P, XROW, &full[s]);
       }
-      const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src));
-      if (ring) *reinterpret_cast<uint4 *>(ring) = raw;
-      const Tin *e = reinterpret_cast<const Tin *>(&raw);
-#pragma unroll
-      for (int c = 0; c < kPer; ++c) dst[c] = to_f32<Tin>(e[c]);
-    }
-    for (int j = tid; j < m; j += kThreads) {
-      const float dtv = to_f32<Tin>(dtin[((size_t)b * m + j) * a.H + h]);
-      s_dt[n + j] = dtv;
-      a.buf2[bh * cap + (st + n + j) % cap] = dtv;
-    }
-    for (int idx = m * N + tid; idx < MAXM * N; idx += kThreads) s_C[idx] = 0.0f;
-  }
-  __syncthreads();
-
-  // 3. Window scalars: a_i = dt_i A, B_i . C_j, coefficients and decays.
-  //    Segment sums are direct sums of the a_r (never ratios of decays).
-  const float Ah = __ldg(a.A + h);
-  for (int i = tid; i < ntot; i += kThreads) s_a[i] = s_dt[i] * Ah;
-  for (int p = warp; p < m * ntot; p += kWarps) {
-    const int j = p / ntot, i = p - j * ntot;
-    if (i < w0 || i > n + j) continue;
-    float acc = 0.0f;
-    for (int c = lane; c < N; c += 32) acc = fmaf(s_B[i * N + c], s_C[j * N + c], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) s_bc[j * cap + i] = acc;
-  }
-  __syncthreads();
-  for (int p = tid; p < m * ntot; p += kThreads) {
-    const int j = p / ntot, i = p - j * ntot, e = n + j;
-    if (i < w0 || i > e) continue;
-    float sg = 0.0f;
-    for (int r = i + 1; r <= e; ++r) sg += s_a[r];
-    s_coef[j * cap + i] = expf(sg) * s_dt[i] * s_bc[j * cap + i];
-  }
-  for (int j = tid; j < m; j += kThreads) {
-    float G = 0.0f;
-    for (int r = w0; r <= n + j; ++r) G += s_a[r];
-    s_dec[j] = expf(G);
-  }
-  if (pre) {
-    for (int i = tid; i < n; i += kThreads) {
-      float sg = 0.0f;
-      for (int r = i + 1; r < n; ++r) sg += s_a[r];
-      s_fwpre[i] = expf(sg) * s_dt[i];
-    }
-    if (tid == 0) {
-      float G = 0.0f;
-      for (int r = 0; r < n; ++r) G += s_a[r];
-      s_dec[MAXM] = expf(G);
-    }
-  }
-  if (post) {
-    for (int i = w0 + tid; i <= n; i += kThreads) {
-      float sg = 0.0f;
-      for (int r = i + 1; r <= n; ++r) sg += s_a[r];
-      s_fwpost[i] = expf(sg) * s_dt[i];
-    }
-    if (tid == 0) {
-      float G = 0.0f;
-      for (int r = w0; r <= n; ++r) G += s_a[r];
-      s_dec[MAXM + 1] = expf(G);
-    }
-  }
-  __syncthreads();
-
-  // 4. New tokens do not fit: fold the committed window into the checkpoint
-  //    first; its read copy is rebuilt from the folded fp32 values.
-  if (pre) {
-    fold_tile<P, N>(st4, s_fwpre, s_dec[MAXM], 0, n, s_x, s_B, row0, c0);
-#pragma unroll
-    for (int l = 0; l < T::NLD; ++l) {
-      const int row = row0 + l * T::RPI;
-      if constexpr (RF != RSSM_READ_FP32)
-        view[l] = quantize4<RF, T::LPR>(st4[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
-      if (!post) st_stream(hc + (size_t)row * N + c0, st4[l]);
-    }
-  }
-
-  // 5. Outputs of the new tokens, from the read view of the checkpoint.
-  if (m > 0) {
-    if constexpr (RF == RSSM_READ_FP32)
-      outputs<P, N, MAXM>(st4, a, s_C, s_x, s_coef, s_dec, b, h, n, w0, warp, lane, c0);
-    else
-      outputs<P, N, MAXM>(view, a, s_C, s_x, s_coef, s_dec, b, h, n, w0, warp, lane, c0);
-  }
-
-  // 6. The decode filled the window: fold all of it.
-  if (post) {
-    fold_tile<P, N>(st4, s_fwpost, s_dec[MAXM + 1], w0, n + 1, s_x, s_B, row0, c0);
-#pragma unroll
-    for (int l = 0; l < T::NLD; ++l) {
-      const int row = row0 + l * T::RPI;
-      st_stream(hc + (size_t)row * N + c0, st4[l]);
-      if constexpr (RF != RSSM_READ_FP32)
-        quantize4<RF, T::LPR>(st4[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
-    }
-  }
-
-  // 7. The last CTA of sequence b moves its pointers.
-  __syncthreads();
-  if (last_arrival(a.arrivals + b, a.H)) {
-    int st2 = st, n2 = n, fl = a.flushes[b];
-    if (pre) {
-      st2 = (st + n) % cap;
-      n2 = 0;
-      ++fl;
-    }
-    if (a.mode == kDecode) {
-      n2 += 1;
-      if (post) {
-        st2 = (st2 + n2) % cap;
-        n2 = 0;
-        ++fl;
+      *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
+      ++jh;
+      if (++s == stages) {
+        s = 0;
+        ++u;
       }
-    } else if (a.mode == kVerify) {
-      a.pending[b] = m;
     }
-    a.start[b] = st2;
-    a.len[b] = n2;
-    a.flushes[b] = fl;
+    if (*abort) {   // let requested copies land (bounded) before the CTA can retire
+      for (int q = issued - stages > 0 ? issued - stages : 0; q < issued; ++q)
+        mbar_wait_bounded(&full[q % stages], (uint32_t)((q / stages) & 1), nullptr, 200000000LL);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int gi = warp / kGroupWarps, gw = warp % kGroupWarps, gt = tid - gi * kGroupThreads;
+  const int bar_id = 1 + gi;
+  float *sB = reinterpret_cast<float *>(smem + stages * stage_bytes) + gi * group_floats;  // [WMAX][N]
+  float *sC = sB + WMAX * N;                                           // [MAXM][N]
+  float *sdt = sC + MAXM * N;                                          // [hc][WMAX]
+  float *sBC = sdt + hc * WMAX;                                        // [MAXM][WMAX]
+  float *ssc = sBC + MAXM * WMAX;                                      // [hc][HS]
+  const int row0 = gw * T::RPW + lane / T::LPR;
+  const int c0 = (lane % T::LPR) * 4;
+  for (int k = gi; k < my_items; k += kGroups) {
+    int b, g, chunk;
+    item_of(k, b, g, chunk);
+    const int h0 = g * a.hpg + chunk * hc;
+    const size_t bh0 = (size_t)b * a.H + h0;
+    Tin *Bring = reinterpret_cast<Tin *>(a.buf1) + ((size_t)b * a.G + g) * cap * N;
+    const RowPlan rp = plan_row(a, b);
+    const int st = rp.st, n = rp.n;
+    const bool pre = rp.pre, post = rp.post;
+    if (rp.refuse && rp.bit && g == 0 && chunk == 0 && gt == 0) atomicOr(a.status, rp.bit);
+    const int w0 = pre ? n : 0;
+    const int ntot = n + m;
+
+    if (!rp.refuse) {
+      // ---- group data: B window and C rows (fp32), dt windows, ring appends
+      constexpr int kPer = 16 / sizeof(Tin);
+      for (int idx = gt; idx < ntot * (N / kPer); idx += kGroupThreads) {
+        const int i = idx / (N / kPer), c = (idx - i * (N / kPer)) * kPer;
+        const Tin *src = i < n ? Bring + (size_t)((st + i) % cap) * N + c
+                               : Bin + (((size_t)b * m + (i - n)) * a.G + g) * N + c;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src));
+        const Tin *e = reinterpret_cast<const Tin *>(&raw);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) sB[i * N + c + q] = to_f32<Tin>(e[q]);
+        if (i >= n && chunk == 0)
+          *reinterpret_cast<uint4 *>(Bring + (size_t)((st + i) % cap) * N + c) = raw;
+      }
+      for (int idx = gt; idx < MAXM * N; idx += kGroupThreads) {
+        const int j = idx / N, c = idx - j * N;
+        sC[idx] = j < m ? to_f32<Tin>(Cin[(((size_t)b * m + j) * a.G + g) * N + c]) : 0.0f;
+      }
+      for (int idx = gt; idx < hc * ntot; idx += kGroupThreads) {
+        const int jh = idx / ntot, i = idx - jh * ntot;
+        const size_t bh = bh0 + jh;
+        float v;
+        if (i < n) {
+          v = a.buf2[bh * cap + (st + i) % cap];
+        } else {
+          v = to_f32<Tin>(dtin[((size_t)b * m + (i - n)) * a.H + h0 + jh]);
+          a.buf2[bh * cap + (st + i) % cap] = v;
+        }
+        sdt[jh * WMAX + i] = v;
+      }
+      for (int idx = gt; idx < hc * m * (P / kPer); idx += kGroupThreads) {
+        const int jh = idx / (m * (P / kPer)), r = idx - jh * (m * (P / kPer));
+        const int j = r / (P / kPer), c = (r - j * (P / kPer)) * kPer;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(xin + (((size_t)b * m + j) * a.H + h0 + jh) * P + c));
+        *reinterpret_cast<uint4 *>(xring + ((bh0 + jh) * cap + (st + n + j) % cap) * P + c) = raw;
+      }
+      named_sync(bar_id, kGroupThreads);
+      for (int p = gw; p < m * ntot; p += kGroupWarps) {
+        const int j = p / ntot, i = p - j * ntot;
+        if (i < w0 || i > n + j) continue;
+        float acc = 0.0f;
+        for (int c = lane; c < N; c += 32) acc = fmaf(sB[i * N + c], sC[j * N + c], acc);
+        acc = warp_sum(acc);
+        if (lane == 0) sBC[j * WMAX + i] = acc;
+      }
+      named_sync(bar_id, kGroupThreads);
+      // ---- window scalars of every head: per (head, task) one warp.  Output j:
+      //      coef_ji = e^{A seg(i, e_j)} dt_i (B_i . C_j) for i in [w0, e_j] (0
+      //      after e_j), dec_j = e^{A G_j}.  Folds: weights e^{A seg(i, last)} dt_i.
+      //      Segment sums are warp suffix sums of the dt (direct sums).
+      for (int t = gw; t < hc * (MAXM + 2); t += kGroupWarps) {
+        const int jh = t / (MAXM + 2), task = t - jh * (MAXM + 2);
+        float *hs = ssc + jh * HS;
+        int i0, len;
+        if (task < MAXM) {
+          if (task >= m) {   // unused output slot: zero coefficients and decay
+            hs[task * 32 + lane] = 0.0f;
+            if (lane == 0) hs[MAXM * 32 + task] = 0.0f;
+            continue;
+          }
+          i0 = w0; len = n + task - w0 + 1;
+        } else if (task == MAXM) {
+          if (!pre) continue;
+          i0 = 0; len = n;
+        } else {
+          if (!post) continue;
+          i0 = w0; len = n - w0 + 1;
+        }
+        const float Ah = __ldg(a.A + h0 + jh);
+        const float v = lane < len ? sdt[jh * WMAX + i0 + lane] : 0.0f;
+        float after, total;
+        suffix_scan(v, lane, after, total);
+        const float wgt = expf(Ah * after) * v;
+        if (task < MAXM) {
+          hs[task * 32 + lane] = lane < len ? wgt * sBC[task * WMAX + i0 + lane] : 0.0f;
+          if (lane == 0) hs[MAXM * 32 + task] = expf(Ah * total);
+        } else {
+          const int q = task - MAXM;
+          hs[MAXM * 32 + MAXM + q * 32 + lane] = wgt;
+          if (lane == 0) hs[MAXM * 32 + MAXM + 64 + q] = expf(Ah * total);
+        }
+      }
+      named_sync(bar_id, kGroupThreads);
+    }
+
+    // ---- heads: every warp of the group works on its rows
+    int s = (k * hc) % stages;
+    int use = (k * hc) / stages;
+    // wait until the producer has requested use `use` of stage s, then for the data
+    auto wait_stage = [&]() -> bool {
+      if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
+      return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
+    };
+    for (int jh = 0; jh < hc; ++jh) {
+      const int h = h0 + jh;
+      if (rp.refuse) {
+        if (!wait_stage()) break;
+      } else {
+        const size_t bh = bh0 + jh;
+        float *hc_tile = a.hc + bh * P * N;
+        uint8_t *rc = (RF != RSSM_READ_FP32) ? a.rc_codes + bh * TB : nullptr;
+        const float *hs = ssc + jh * HS;
+        const float *hcoef = hs, *hdec = hs + MAXM * 32, *hfw = hs + MAXM * 32 + MAXM;
+        const float *hdecf = hfw + 64;
+        float4 f[T::NLD];   // fp32 checkpoint values for a fold (read-copy layers)
+        if constexpr (RF != RSSM_READ_FP32) {
+          if (pre || post) {
+#pragma unroll
+            for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_tile + (size_t)(row0 + l * T::RPI) * N + c0);
+          }
+        }
+        if (!wait_stage()) break;
+        const Stage stg{smem + s * stage_bytes, XOFF, XROW, n, L};
+
+        float4 v[T::NLD];
+        if (pre) {   // the new tokens do not fit: fold the committed window first
+          if constexpr (RF == RSSM_READ_FP32) {
+#pragma unroll
+            for (int l = 0; l < T::NLD; ++l)
+              f[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(row0 + l * T::RPI) * N + c0) * 4);
+          }
+          fold_tile<P, N, kGroupWarps, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
+#pragma unroll
+          for (int l = 0; l < T::NLD; ++l) {
+            const int row = row0 + l * T::RPI;
+            if (!post) st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+            if constexpr (RF == RSSM_READ_FP32)
+              v[l] = f[l];
+            else
+              v[l] = quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+          }
+        } else {
+#pragma unroll
+          for (int l = 0; l < T::NLD; ++l) {
+            const int row = row0 + l * T::RPI;
+            if constexpr (RF == RSSM_READ_FP32) {
+              v[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)row * N + c0) * 4);
+            } else if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+              const uint32_t w = *reinterpret_cast<const uint32_t *>(stg.base + (size_t)row * RB + c0);
+              dec_e4m3x4(w, reinterpret_cast<const float *>(stg.base + TB)[row], v[l]);
+            } else {
+              const uint32_t w = *reinterpret_cast<const uint16_t *>(stg.base + (size_t)row * RB + c0 / 2);
+              const float sc = dec_e4m3(stg.base[TB + row * (N / 16) + c0 / 16]);
+              dec_e2m1x4(w, sc, v[l]);
+            }
+          }
+        }
+        if (m > 0)
+          outputs<P, N, kGroupWarps, Tin, MAXM>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
+        if (post) {  // the decode filled the window: fold all of it
+          if constexpr (RF == RSSM_READ_FP32) {
+#pragma unroll
+            for (int l = 0; l < T::NLD; ++l) f[l] = v[l];
+          }
+          fold_tile<P, N, kGroupWarps, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
+#pragma unroll
+          for (int l = 0; l < T::NLD; ++l) {
+            const int row = row0 + l * T::RPI;
+            st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+            if constexpr (RF != RSSM_READ_FP32)
+              quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);   // this warp is done with stage s
+      if (++s == stages) {
+        s = 0;
+        ++use;
+      }
+    }
+
+    // ---- item end: the group's warps are done; the last CTA of sequence b
+    //      moves its pointers.  An abort stops the group here.
+    const bool any_abort = named_sync_or(bar_id, kGroupThreads, *abort != 0);
+    if (any_abort) {
+      if (gt == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
+      return;
+    }
+    if (!rp.refuse && gt == 0) {
+      __threadfence();
+      if (atomicAdd(a.arrivals + b, 1) == a.G * nchunk - 1) {
+        a.arrivals[b] = 0;
+        int st2 = st, n2 = n, fl = a.flushes[b];
+        if (pre) {
+          st2 = (st + n) % cap;
+          n2 = 0;
+          ++fl;
+        }
+        if (a.mode == kDecode) {
+          n2 += 1;
+          if (post) {
+            st2 = (st2 + n2) % cap;
+            n2 = 0;
+            ++fl;
+          }
+        } else if (a.mode == kVerify) {
+          a.pending[b] = m;
+        }
+        a.start[b] = st2;
+        a.len[b] = n2;
+        a.flushes[b] = fl;
+      }
+    }
   }
 }
 
@@ -398,20 +614,44 @@ __global__ void __launch_bounds__(kThreads) m2_conv_kernel(const ConvArgs a) {
   }
 }
 
-size_t step_smem_bytes(int P, int N, int cap, int maxm) {
-  return sizeof(float) * ((size_t)cap * (P + N) + (size_t)maxm * N + 2 * (size_t)cap +
-                          2 * (size_t)maxm * cap + 2 * (size_t)cap + maxm + 2);
+int heads_per_cta(int hpg) {
+  int hc = hpg < 16 ? hpg : 16;
+  while (hpg % hc) --hc;
+  return hc;
 }
 
 template <int P, int N, typename Tin, int RF, int MAXM>
 cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
-  auto kern = m2_step_kernel<P, N, Tin, RF, MAXM>;
-  const size_t smem = step_smem_bytes(P, N, a.cap, MAXM);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  kern<<<dim3((unsigned)(a.B * a.H)), dim3(kThreads), smem, s>>>(a);
+  auto kern = m2_replay_kernel<P, N, Tin, RF, MAXM>;
+  const int hc = heads_per_cta(a.hpg);
+  const size_t xrow = (size_t)P * sizeof(Tin);
+  const size_t stage = ((size_t)tile_bytes<RF, P, N>() + scale_bytes<RF, P, N>() + (a.L + MAXM) * xrow + 127) & ~(size_t)127;
+  const size_t wmax = a.L + MAXM;
+  const size_t group_floats = (wmax * N + MAXM * N + hc * wmax + MAXM * wmax +
+                               (size_t)hc * (MAXM * 32 + MAXM + 64 + 2) + 31) & ~(size_t)31;
+  const size_t fixed = kGroups * sizeof(float) * group_floats;
+  // One CTA per SM (its 544 threads use the register file); as many stages as
+  // fit in its shared memory, at most 5 for fp32 tiles (32 KiB each) and
+  // kMaxStages for the smaller read-copy tiles.
+  int dev = 0, sms = 0, max_smem = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  const size_t budget = (size_t)max_smem - 2048;
+  if (fixed + 2 * stage > budget) return cudaErrorInvalidConfiguration;
+  int stages = (int)((budget - fixed) / stage);
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (RF == RSSM_READ_FP32 && stages > 5) stages = 5;
+  const size_t smem = fixed + (size_t)stages * stage;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+  int per_sm = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kReplayThreads, smem)) != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const long long items = (long long)a.B * a.G * (a.hpg / hc);
+  const long long slots = (long long)sms * per_sm;
+  const unsigned grid = (unsigned)(items < slots ? items : slots);
+  kern<<<dim3(grid), dim3(kReplayThreads), smem, s>>>(a, hc, stages);
   return cudaGetLastError();
 }
 

@@ -64,13 +64,14 @@ enum {
   RSSM_ERR_CAPACITY = 3,    /* more drafts than the window can hold        */
   RSSM_ERR_STATE = 4,       /* call not valid in the handle's state        */
   RSSM_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed        */
-  RSSM_ERR_TIMEOUT = 6      /* reserved: a bounded device wait gave up     */
+  RSSM_ERR_TIMEOUT = 6      /* reserved for host-side waits                */
 };
 
 /* Sticky device status bits (rssm_get_status). */
 enum {
   RSSM_STATUS_CAPACITY = 1u << 0, /* row could not append: window full, auto_flush off */
-  RSSM_STATUS_STATE = 1u << 1     /* row refused: drafts pending / bad rollback count  */
+  RSSM_STATUS_STATE = 1u << 1,    /* row refused: drafts pending / bad rollback count  */
+  RSSM_STATUS_TIMEOUT = 1u << 2   /* a bounded wait for an asynchronous copy gave up   */
 };
 
 enum { RSSM_MAMBA2 = 1, RSSM_GDN = 2 };

@@ -296,3 +296,42 @@ def test_read_copy_keeps_fp32_recurrence(fmt):
         if book.decode()[0][3]:
             h_ckpt = h_exact.copy()
             window_toks = []
+
+
+@pytest.mark.parametrize("fmt", [rssm.RSSM_READ_FP32, rssm.RSSM_READ_FP8_E4M3_ROW, rssm.RSSM_READ_NVFP4])
+def test_many_items_per_cta(fmt):
+    """One head per group (G = H) and enough sequences that every persistent CTA
+    works through several items, so the copies requested ahead cross item
+    boundaries; verify rounds with ragged acceptance make rows fold at
+    different calls of the same launch."""
+    shape = si.Mamba2Layer(batch=96, nheads=8, headdim=64, dstate=128, ngroups=8, window=6,
+                           dtype="bf16", state_std=0.1, max_draft=3)
+    layer, A, D, h0 = m2_layer(shape, read_fmt=fmt)
+    h = h0.double().numpy()
+    book = ob.WindowBook(96, 6, int(layer.layout.cap))
+    yk = torch.empty(96, 3, 8, 64, device=DEV)
+    y = torch.empty(96, 8, 64, device=DEV)
+    for r in range(8):
+        drafts = si.mamba2_drafts(shape, r, 3, seed=5)
+        acc = si.accept_counts(96, r, 3, seed=5)
+        layer.verify(3, dev_inputs(drafts, M2_KEYS), yk)
+        book.verify(3)
+        want, h_next = osp.mamba2_round(h, tok64(drafts), acc.numpy(), A, D)
+        if fmt == rssm.RSSM_READ_FP32:
+            assert_close(yk.cpu(), want, TOL["bf16"], f"verify round {r}")
+        else:   # low-precision reads: bounded by the quantisation, checked elsewhere
+            assert rel_err(yk.cpu(), want) < (0.1 if fmt == rssm.RSSM_READ_FP8_E4M3_ROW else 0.5)
+        n_reject = (3 - acc).to(torch.int32)
+        layer.rollback(n_reject.to(DEV))
+        book.rollback(n_reject.tolist())
+        h = h_next
+        tok = si.mamba2_tokens(shape, 500 + r, seed=5)
+        layer.decode_step(dev_inputs(tok, M2_KEYS), y)
+        book.decode()
+        h, yy = _oracle_step(h, tok, A, D)
+        assert _bk(layer) == [list(x) for x in book.snapshot()]
+    layer.flush()
+    book.flush()
+    assert_close(layer.ckpt.cpu(), h, TOL["bf16"], "checkpoint")
+    assert _bk(layer) == [list(x) for x in book.snapshot()]
+    assert layer.get_status() == 0
