@@ -341,3 +341,70 @@ const char *rssm_last_error_string(void) { return g_err.c_str(); }
 uint64_t rssm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode step with library-owned scratch (rssm_decode_step_static_scratch).
+//
+// The replay kernel needs one int32 arrival counter per sequence: the CTAs of a
+// sequence count themselves in, and the last one moves the ring pointers.
+// rssm_decode_step keeps those counters in the caller's meta buffer.  Some
+// callers cannot hand the library any memory beyond the layer's own buffers
+// at call time: code that records decode steps into a CUDA graph (no
+// allocation may happen inside the capture), serving engines that reserve all
+// device memory up front and forbid later cudaMalloc, and latency-critical
+// loops that must avoid cudaMalloc's implicit device synchronisation.  For
+// them the counters below live in a fixed array in the library's own device
+// image, so the call allocates nothing.
+namespace {
+
+static __device__ __align__(256) int32_t g_static_arrivals[RSSM_STATIC_SCRATCH_MAX_BATCH];
+
+constexpr int kMaxDevices = 64;
+std::atomic<int32_t *> g_static_arrivals_dev[kMaxDevices];
+
+// Device address of g_static_arrivals for the current device (host code may
+// not use the symbol itself as an address).  Looked up once per device.
+int static_arrivals_for_current_device(int32_t **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RSSM_ERR_UNSUPPORTED, "device index %d too large", dev);
+  int32_t *p = g_static_arrivals_dev[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_static_arrivals);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_static_arrivals)");
+    g_static_arrivals_dev[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return RSSM_OK;
+}
+
+}  // namespace
+
+extern "C" int rssm_decode_step_static_scratch(rssm_handle *h, const void *const *in, void *out_dev,
+                                               rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.batch > RSSM_STATIC_SCRATCH_MAX_BATCH)
+    return fail(RSSM_ERR_INVALID_ARG,
+                "batch %d exceeds the %d sequences the library's static scratch holds; "
+                "use rssm_decode_step",
+                h->d.batch, RSSM_STATIC_SCRATCH_MAX_BATCH);
+  int rc = check_inputs(h, in, out_dev);
+  if (rc) return rc;
+  int32_t *arrivals = nullptr;
+  rc = static_arrivals_for_current_device(&arrivals);
+  if (rc) return rc;
+  // The counters must start at zero; a previous call leaves them at zero unless
+  // it was cut short, so clear the ones this call uses.
+  cudaError_t e = cudaMemsetAsync(arrivals, 0, sizeof(int32_t) * (size_t)h->d.batch, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(static scratch)");
+  rssm::StepArgs a = step_args(h, rssm::kDecode, 1);
+  for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
+  a.out = static_cast<float *>(out_dev);
+  a.arrivals = arrivals;
+  e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream)
+                               : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");
+  return ok();
+}

@@ -32,7 +32,9 @@ EXPORTED = [
     "rssm_decode_step", "rssm_verify", "rssm_rollback", "rssm_flush",
     "rssm_quantize_read_copy", "rssm_conventional_step", "rssm_get_bookkeeping",
     "rssm_get_status", "rssm_last_error_string", "rssm_launch_count",
+    "rssm_decode_step_static_scratch",
 ]
+RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
 
 class LayerDesc(C.Structure):
@@ -70,6 +72,7 @@ def lib():
         L.rssm_set_params.argtypes = [vp, vp, vp]
         L.rssm_decode_step.argtypes = [vp, C.POINTER(vp), vp, vp]
         L.rssm_verify.argtypes = [vp, i32, C.POINTER(vp), vp, vp]
+        L.rssm_decode_step_static_scratch.argtypes = [vp, C.POINTER(vp), vp, vp]
         L.rssm_rollback.argtypes = [vp, vp, vp]
         L.rssm_flush.argtypes = [vp, vp, vp]
         L.rssm_quantize_read_copy.argtypes = [vp, vp]

@@ -227,6 +227,29 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev,
                            float *state_out_dev, const void *const *in,
                            void *out_dev, rssm_stream_t stream);
 
+/*
+ * rssm_decode_step without any caller-provided scratch.  (This entry point has
+ * no counterpart on the pages; it serves integration needs only.)
+ *
+ * Identical inputs, outputs and results to rssm_decode_step.  The replay
+ * kernel's only scratch -- one int32 arrival counter per sequence -- comes
+ * from a fixed array inside the library (RSSM_STATIC_SCRATCH_MAX_BATCH
+ * entries, 256 KiB on every GPU that loads the library, kept until the
+ * process exits) instead of the caller's meta buffer, so the call performs
+ * no allocation: for callers that record decode steps into a CUDA graph,
+ * engines that reserve all device memory at start-up, and loops that cannot
+ * afford cudaMalloc's implicit synchronisation.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Each call clears the counters it uses (cudaMemsetAsync on `stream`).
+ *   - All calls share the one array: calls that may run concurrently on the
+ *     GPU (different streams, different handles) race and must not overlap.
+ *   - batch > RSSM_STATIC_SCRATCH_MAX_BATCH: RSSM_ERR_INVALID_ARG.
+ */
+#define RSSM_STATIC_SCRATCH_MAX_BATCH 65536
+int rssm_decode_step_static_scratch(rssm_handle *h, const void *const *in,
+                                    void *out_dev, rssm_stream_t stream);
+
 /* Copy the per-sequence pointers into out_dev (device int32 [4, B]: start,
  * len, pending, flushes). */
 int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev,
