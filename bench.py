@@ -221,7 +221,59 @@ class Mamba2Work:
         return time.perf_counter() - t0
 
 
-WORKLOADS = {"mamba2": Mamba2Work}
+class GDNWork:
+    name = "gdn"
+    keys = ("q", "k", "v", "alpha", "beta")
+    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/gdn.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
+
+    def __init__(self, dev, seed, batch=None):
+        from hybrid_ssm_decode_replayssm_b200 import rssm
+        self.shape = s = si.GDN_SERVING if batch is None else si.GDN_SERVING.with_(batch=batch)
+        self.h0 = si.gdn_checkpoint(s, seed).to(dev)
+        self.desc = rssm.make_desc(rssm.RSSM_GDN, s.batch, s.nheads, s.dv, s.dk, window=s.window,
+                                   max_draft=s.max_draft, in_dtype=rssm.RSSM_BF16)
+        self.host_pool = [si.gdn_tokens(s, t, seed) for t in range(POOL)]
+        self.pool = [[tok[k].to(dev) for k in self.keys] for tok in self.host_pool]
+        self.out_shape = (s.batch, s.nheads, s.dv)
+        self.tokens_per_call = s.batch
+        self.workload = (f"Gated DeltaNet decode layer: batch {s.batch}, {s.nheads} heads, d_k = d_v = {s.dk}, "
+                         f"bf16 q/k/v, fp32 alpha/beta, fp32 checkpoint, L={s.window}")
+
+    def layer(self):
+        from hybrid_ssm_decode_replayssm_b200 import rssm
+        return rssm.ReplayLayer(self.desc, self.h0.clone())
+
+    def bytes_per_call(self, pos):
+        """Algorithmic bytes of the decode call at window position pos (1..L)."""
+        s = self.shape
+        BH, dk, dv, L = s.batch * s.nheads, s.dk, s.dv, s.window
+        ck = BH * dv * dk * 4
+        inputs = BH * (2 * dk + dv) * 2 + BH * 8                     # q, k, v, alpha, beta
+        append = BH * (dk + dv) * 2 + BH * 8 + BH * dv * 4            # k, v, g, beta rows; new w
+        entry = BH * dk * 2 + BH * dv * 4 + BH * 8                    # k, w, g, beta per window entry
+        out = BH * dv * 4
+        fold = ck + (L - 1) * BH * dv * 2 if pos == L else 0          # state write; v rows re-read
+        return ck + inputs + append + (pos - 1) * entry + out + fold
+
+    def conventional_bytes(self):
+        s = self.shape
+        BH = s.batch * s.nheads
+        return 2 * BH * s.dv * s.dk * 4 + BH * (2 * s.dk + s.dv) * 2 + BH * 8 + BH * s.dv * 4
+
+    def oracle_sample(self, nseq, steps, seed):
+        """Time the fp64 oracle (conventional gated delta rule) on nseq sequences x all heads."""
+        from oracle import gdn as og
+        S = self.h0[:nseq].double().cpu().numpy()
+        toks = [{k: v[:nseq].double().numpy() for k, v in self.host_pool[t % POOL].items()} for t in range(steps)]
+        t0 = time.perf_counter()
+        for tok in toks:
+            S, _ = og.step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+        return time.perf_counter() - t0
+
+
+WORKLOADS = {"mamba2": Mamba2Work, "gdn": GDNWork}
 
 
 # ------------------------------------------------------------------ timing

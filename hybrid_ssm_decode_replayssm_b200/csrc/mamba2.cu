@@ -49,21 +49,6 @@ constexpr int scale_bytes() {
 template <int RF, int N>
 constexpr int rc_row_bytes() { return RF == RSSM_READ_NVFP4 ? N / 2 : N; }
 
-// Suffix sums over a warp: lanes l < len hold v (the others 0).  Returns in
-// `after` the sum of v over lanes l' > l (direct sums of the terms, no
-// differences of prefix sums) and in `total` the sum over all lanes.
-__device__ __forceinline__ void suffix_scan(float v, int lane, float &after, float &total) {
-  float incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float t = __shfl_down_sync(kFull, incl, o);
-    if (lane + o < 32) incl += t;
-  }
-  after = __shfl_down_sync(kFull, incl, 1);
-  if (lane == 31) after = 0.0f;
-  total = __shfl_sync(kFull, incl, 0);
-}
-
 // Stage layout for one head: [read tile | scales | committed x rows (L) | new x rows (MAXM)].
 struct Stage {
   uint8_t *base;

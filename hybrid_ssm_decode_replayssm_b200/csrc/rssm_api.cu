@@ -88,11 +88,11 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
     L->buf_off[1] = off; off = align256(off + B * G * cap * C * esz);      // B_buf
     L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // dt_buf
   } else {
-    L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf
-    L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf
-    L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // g_buf
-    L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf
-    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf
+    L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf [B,H,cap,dk]
+    L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf [B,H,2,cap,dv/2]
+    L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // g_buf [B,H,cap]
+    L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf [B,H,cap]
+    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf [B,H,2,cap,dv/2]
   }
   *buf = off;
   if (d->read_fmt == RSSM_READ_FP32) {

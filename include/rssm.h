@@ -114,9 +114,11 @@ typedef struct {
  * cap = window + max(max_draft, 1) is the ring capacity per sequence.
  *   buf, Mamba-2: x_buf [B,H,cap,P] in_dtype | B_buf [B,G,cap,N] in_dtype |
  *                 dt_buf [B,H,cap] fp32
- *   buf, GDN:     k_buf [B,H,cap,dk] in_dtype | v_buf [B,H,cap,dv] in_dtype |
+ *   buf, GDN:     k_buf [B,H,cap,dk] in_dtype | v_buf [B,H,2,cap,dv/2] in_dtype
+ *                 (value rows split in two halves, half-major) |
  *                 g_buf [B,H,cap] fp32 (ln alpha) | beta_buf [B,H,cap] fp32 |
- *                 w_buf [B,H,cap,dv] fp32 (solved w_s, a cache for reads)
+ *                 w_buf [B,H,2,cap,dv/2] fp32 (solved w_s, half-major; a cache
+ *                 for reads, never used by a fold)
  *   read copy, FP8 row: codes [B,H,R,C] uint8 | scales [B,H,R] fp32
  *   read copy, NVFP4:   codes [B,H,R,C/2] uint8 (element 2i in the low
  *                       nibble) | scales [B,H,R,C/16] uint8 (E4M3)
