@@ -465,7 +465,9 @@ def main():
                 "peak_source": f"{peak_kind} copy bandwidth",
                 "kernel": f"{work.name} replay decode (append + output, fold every {L}th call)",
                 "bytes_per_launch_avg": alg_bytes / len(per),
-                "launch_us_avg": round(kern_time / len(per) * 1e6, 2)}
+                "launch_us_avg": round(kern_time / len(per) * 1e6, 2),
+                "launch_us_fold": round(statistics.mean(p for p, q in zip(per, positions) if q == L) * 1e6, 2),
+                "launch_us_nofold": round(statistics.mean(p for p, q in zip(per, positions) if q != L) * 1e6, 2)}
 
     conv = None
     if "conventional" in legs:

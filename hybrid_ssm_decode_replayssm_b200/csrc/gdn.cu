@@ -134,19 +134,21 @@ __device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
 // Per-group shared scalars of the current head.
 template <int MAXM>
 struct HeadScalars {
-  static constexpr int kOut = MAXM + 2 * MAXM * 32;             // dec, Mk, Mq
-  static constexpr int kFold = kMaxW + kMaxW * kMaxW + kMaxW + 4; // decf, Mf, fw, decF, 1-entry fold
-  static constexpr int kDots = 2 * MAXM * 32;                   // k.k_e, k.q per output
+  static constexpr int kOut = MAXM + 2 * MAXM * 32;             // per head: dec, Mk, Mq
+  static constexpr int kFold = kMaxW + 2 * kMaxW * kMaxW + kMaxW + 4; // decf, A, T, fw, decF, 1-entry fold
+  static constexpr int kDots = 0;
   static constexpr int kWarp = kMaxW * RPW + 2 * MAXM * RPW;     // U/W fold scratch, reductions
 };
 
 // Fold of the window entries [i0, i0 + nf) into the fp32 rows t (8 rows of this
-// warp, 4 columns of this lane): solve the w_i from t itself (matvecs t k_i in
-// chunks of 4, then forward substitution per row), then
-// t <- decF t + sum_i fw_i w_i k_i^T.   decf_i = e^{G_i}, Mf[i][i'] = e^{seg(i',i)} k_i'.k_i.
+// warp, 4 columns of this lane), by the UT transform of the window: with
+// u_i = t k_i (matvecs in chunks of 4 keys), r_i = beta_i (v_i - e^{G_i} u_i)
+// and T = (I + A)^{-1}, A[i][i'] = beta_i e^{seg(i',i)} k_i'.k_i (i' < i), the
+// solved values are w = T r (forward substitution done once per head in T),
+// then t <- decF t + sum_i fw_i w_i k_i^T.
 template <typename Tin>
 __device__ void fold_rows(float4 (&t)[RPW], const GStage<Tin> &stg, int i0, int nf, const float *decf,
-                          const float *Mf, const float *fw, float decF, const float *beta, int urow0,
+                          const float *Tm, const float *fw, float decF, const float *beta, int urow0,
                           float *U, int lane, int c0) {
   for (int ch = 0; ch < nf; ch += 4) {
     float part[RPW * 4];
@@ -162,14 +164,25 @@ __device__ void fold_rows(float4 (&t)[RPW], const GStage<Tin> &stg, int i0, int 
     if (i < nf) U[i * RPW + r] = part[0];
   }
   __syncwarp();
-  if (lane < RPW) {   // forward substitution, one row per lane
-    const int r = lane;
-    for (int i = 0; i < nf; ++i) {
-      float acc = fmaf(-decf[i], U[i * RPW + r], to_f32<Tin>(stg.v(i0 + i)[urow0 + r]));
-      for (int ip = 0; ip < i; ++ip) acc = fmaf(-Mf[i * kMaxW + ip], U[ip * RPW + r], acc);
-      U[i * RPW + r] = beta[i0 + i] * acc;
-    }
+  for (int p = lane; p < nf * RPW; p += 32) {   // r_i per (entry, row); U[i][r] layout
+    const int i = p / RPW, r = p - i * RPW;
+    U[p] = beta[i0 + i] * fmaf(-decf[i], U[p], to_f32<Tin>(stg.v(i0 + i)[urow0 + r]));
   }
+  __syncwarp();
+  constexpr int kPer = kMaxW * RPW / 32;
+  float wv[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int p = lane + 32 * q, i = p / RPW, r = p - i * RPW;
+    float acc = 0.0f;
+    if (i < nf)
+      for (int ip = 0; ip <= i; ++ip) acc = fmaf(Tm[i * kMaxW + ip], U[ip * RPW + r], acc);
+    wv[q] = acc;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < kPer; ++q)
+    if (lane + 32 * q < nf * RPW) U[lane + 32 * q] = wv[q];
   __syncwarp();
 #pragma unroll
   for (int r = 0; r < RPW; ++r) scale4(t[r], decF);
@@ -208,7 +221,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   const int VOFF = QOFF + MAXM * KROW;
   const int WOFF = VOFF + (L + MAXM) * VHROW;
   const size_t stage_bytes = ((size_t)WOFF + (size_t)L * HALF * 4 + 127) & ~(size_t)127;
-  const int group_floats = (2 * hc * WMAX + HS::kOut + HS::kFold + HS::kDots + kGroupWarps * HS::kWarp + 31) & ~31;
+  const int group_floats = (2 * hc * WMAX + hc * HS::kOut + HS::kFold + kGroupWarps * HS::kWarp + 31) & ~31;
 
   const Tin *qin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *kin = reinterpret_cast<const Tin *>(a.in[1]);
@@ -240,20 +253,29 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    int cur_k = -1, b = 0, chunk = 0, unit = 0, s = 0, u = 0;
-    RowPlan rp{};
+    // Issue order: the units of items 2p and 2p+1 interleaved (unit u of 2p, unit
+    // u of 2p+1, unit u+1 of 2p, ...), so both consumer groups work at once.
+    int b2[2] = {0, 0}, chunk2[2] = {0, 0}, s = 0, u = 0, cur_pair = -1;
+    RowPlan rp2[2] = {};
     int issued = 0;
     for (int seq = 0; seq < total_seq; ++seq) {
       if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
         atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
         break;
       }
-      if (cur_k < 0 || unit == 2 * hc) {
-        ++cur_k;
-        unit = 0;
-        item_of(cur_k, b, chunk);
-        rp = plan_row(a, b);
+      const int p = seq / (4 * hc), within = seq - p * 4 * hc;
+      const bool paired = 2 * p + 1 < my_items;
+      const int gsel = paired ? (within & 1) : 0;
+      const int unit = paired ? (within >> 1) : within;
+      if (p != cur_pair) {
+        cur_pair = p;
+        for (int g2 = 0; g2 < (paired ? 2 : 1); ++g2) {
+          item_of(2 * p + g2, b2[g2], chunk2[g2]);
+          rp2[g2] = plan_row(a, b2[g2]);
+        }
       }
+      const int b = b2[gsel], chunk = chunk2[gsel];
+      const RowPlan &rp = rp2[gsel];
       issued = seq + 1;
       if (rp.refuse) {
         mbar_arrive(&full[s]);
@@ -262,7 +284,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         const int h = chunk * hc + jh;
         const size_t bh = (size_t)b * a.H + h;
         const bool fold = rp.pre || rp.post;
-        const int nk = (hf == 0 || fold) ? rp.n : 0;   // committed k rows
+        const int nk = fold ? rp.n : 0;                // committed k rows (fold passes)
         const int nv = fold ? rp.n : 0;                // committed v rows
         const int nw = rp.pre ? 0 : rp.n;              // committed w rows
         uint8_t *dst = smem + s * stage_bytes;
@@ -297,7 +319,6 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         }
       }
       *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
-      ++unit;
       if (++s == stages) {
         s = 0;
         ++u;
@@ -316,16 +337,15 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   float *gbase = reinterpret_cast<float *>(smem + stages * stage_bytes) + gi * group_floats;
   float *sg = gbase;                          // [hc][WMAX]  ln alpha
   float *sbeta = sg + hc * WMAX;              // [hc][WMAX]
-  float *hso = sbeta + hc * WMAX;             // dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
-  float *hsf = hso + HS::kOut;                // decf[32] | Mf[32][32] | fw[32] | decF
-  float *hdots = hsf + HS::kFold;             // KK[MAXM][32] | KQ[MAXM][32]
-  float *wscr = hdots + HS::kDots + gw * HS::kWarp;
+  float *hso = sbeta + hc * WMAX;             // per head: dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
+  float *hsf = hso + hc * HS::kOut;           // decf[32] | A[32][32] | T[32][32] | fw[32] | decF | one[3]
+  float *wscr = hsf + HS::kFold + gw * HS::kWarp;
   float *U = wscr, *red = wscr + kMaxW * RPW;
-  float *odec = hso, *Mk = hso + MAXM, *Mq = Mk + MAXM * 32;
-  float *decf = hsf, *Mf = hsf + kMaxW, *fw = Mf + kMaxW * kMaxW, *decF = fw + kMaxW;
+  float *odec = hso, *Mk = hso + MAXM, *Mq = Mk + MAXM * 32;   // repointed per head
+  float *decf = hsf, *Mf = hsf + kMaxW, *Tm = Mf + kMaxW * kMaxW, *fw = Tm + kMaxW * kMaxW;
+  float *decF = fw + kMaxW;
   float *one = decF + 1;   // window-full fold of a 1-entry window after a pre-fold (L = 1):
-                           // one[0] = e^{g} (its decf and decF), one[1] = 1 (its fw)
-  float *KK = hdots, *KQ = hdots + MAXM * 32;
+                           // one[0] = e^{g} (its decf and decF), one[1] = 1 (fw), one[2] = 1 (T)
   const int c0 = lane * 4;
   const int urow0 = gw * RPW;   // first row of this warp inside a unit
 
@@ -381,10 +401,77 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         }
       }
       named_sync(bar_id, kGroupThreads);
+      // ---- output scalars of every head (one warp per head), from the k rows of
+      //      the ring and the inputs: for output j (e = n + j) and window entry
+      //      i in [w0, e]: Mq_ji = e^{seg(i,e)} k_i.q_j, Mk_ji = e^{seg(i,e)} k_i.k_e
+      //      (i < e), 0 elsewhere; dec_j = e^{G}, G the g summed over [w0, e].
+      if (m > 0) {
+        constexpr int CE = MAXM == 1 ? 8 : 4;   // window entries per reduction
+        constexpr int NV = CE * 2 * MAXM;
+        for (int jh = gw; jh < hc; jh += kGroupWarps) {
+          const size_t bh = bh0 + jh;
+          float *hs = hso + jh * HS::kOut;
+          float *hMk = hs + MAXM, *hMq = hMk + MAXM * 32;
+          float4 qv[MAXM], kv[MAXM];
+#pragma unroll
+          for (int j = 0; j < MAXM; ++j) {
+            const size_t tok = ((size_t)b * m + j) * a.H + h0 + jh;
+            qv[j] = j < m ? ld4<Tin>(qin + tok * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+            kv[j] = j < m ? ld4<Tin>(kin + tok * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          for (int i0 = w0; i0 < ntot; i0 += CE) {
+            float part[NV];
+#pragma unroll
+            for (int c = 0; c < CE; ++c) {
+              const int i = i0 + c;
+              float4 ki = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (i < n)
+                ki = ld4<Tin>(kring + (bh * cap + (st + i) % cap) * DK + c0);
+              else if (i < ntot)
+                ki = ld4<Tin>(kin + (((size_t)b * m + (i - n)) * a.H + h0 + jh) * DK + c0);
+#pragma unroll
+              for (int j = 0; j < MAXM; ++j) {
+                part[(c * MAXM + j) * 2 + 0] = dot4(ki, qv[j]);
+                part[(c * MAXM + j) * 2 + 1] = dot4(ki, kv[j]);
+              }
+            }
+            tr_sum<NV, 16>(part, lane);
+            const int base = tr_base<NV, 16>(lane);
+            constexpr int R = NV >= 32 ? NV / 32 : 1;
+            constexpr int DUP = NV >= 32 ? 1 : 32 / NV;
+            if ((lane & (DUP - 1)) == 0) {
+#pragma unroll
+              for (int q = 0; q < R; ++q) {   // raw dots, scaled below by their decays
+                const int idx = base + q, which = idx & 1, j = (idx >> 1) % MAXM, c = (idx >> 1) / MAXM;
+                const int l = i0 - w0 + c;
+                if (l < 32) (which == 0 ? hMq : hMk)[j * 32 + l] = part[q];
+              }
+            }
+          }
+          __syncwarp();
+          const int l = lane, i = w0 + l;
+#pragma unroll
+          for (int j = 0; j < MAXM; ++j) {
+            const int e = n + j, len = e - w0 + 1;
+            const float v = (j < m && l < len) ? sg[jh * WMAX + i] : 0.0f;
+            float after, total;
+            suffix_scan(v, lane, after, total);
+            const float ex = expf(after);
+            const bool in = j < m && l < len;
+            hMq[j * 32 + l] = in ? ex * hMq[j * 32 + l] : 0.0f;
+            hMk[j * 32 + l] = (in && l < len - 1) ? ex * hMk[j * 32 + l] : 0.0f;
+            if (lane == 0) hs[j] = j < m ? expf(total) : 0.0f;
+          }
+        }
+      }
+      named_sync(bar_id, kGroupThreads);
     }
 
-    int s = (k * hc * 2) % stages;
-    int use = (k * hc * 2) / stages;
+    // sequence number of this item's unit `unit` in the producer's issue order
+    const int pair = k >> 1;
+    const bool paired = 2 * pair + 1 < my_items;
+    const int seq0 = pair * 4 * hc + (paired ? (k & 1) : 0), step = paired ? 2 : 1;
+    int s = seq0 % stages, use = seq0 / stages;   // stage and use of the current unit
     auto wait_stage = [&]() -> bool {
       if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
       return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
@@ -392,8 +479,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     auto release_stage = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == stages) {
-        s = 0;
+    };
+    auto next_unit = [&]() {
+      s += step;
+      if (s >= stages) {
+        s -= stages;
         ++use;
       }
     };
@@ -406,7 +496,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       const int h = h0 + jh;
       const size_t bh = bh0 + jh;
       const float *gw_ = sg + jh * WMAX, *bw_ = sbeta + jh * WMAX;
-      for (int hf = 0; hf < 2; ++hf) {
+      odec = hso + jh * HS::kOut;
+      Mk = odec + MAXM;
+      Mq = Mk + MAXM * 32;
+      for (int hf = 0; hf < 2; ++hf, next_unit()) {
         if (rp.refuse) {
           if (!failed && wait_stage()) release_stage();
           else failed = true;
@@ -422,73 +515,70 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             for (int r = 0; r < RPW; ++r) f[r] = ld_stream(hc_rows + (size_t)(urow0 + r) * DK + c0);
           }
         }
-        if (hf == 0 && named_sync_or(bar_id, kGroupThreads, failed)) failed = true;  // scalars free
+        // fold scalars are single-buffered: all warps must be done with the previous head's
+        if (hf == 0 && (pre || post) && named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
         const bool have = !failed && wait_stage();
         if (!have) failed = true;
         const GStage<Tin> stg{smem + s * stage_bytes, KOFF, QOFF, VOFF, WOFF, n, L};
 
-        if (hf == 0) {
-          // ---- head scalars.  Dots: output j (e = n + j): k_i.q_j for i in
-          //      [w0, e], k_i.k_e for i in [w0, e); fold: k_i'.k_i, i' < i.
-          const int nout = m > 0 ? (n + m - w0) * 2 * m : 0;
-          const int nfold = (pre || post) ? nf * nf : 0;
-          for (int t = gw; have && t < nout + nfold; t += kGroupWarps) {
-            float *dst;
-            const Tin *ra, *rb;
-            if (t < nout) {
-              const int j = t / (2 * (n + m - w0)), rem2 = t - j * 2 * (n + m - w0);
-              const int which = rem2 & 1, l = rem2 >> 1, i = w0 + l, e = n + j;
-              if (j >= m || i > e || (which == 1 && i == e)) continue;
-              ra = stg.k(i);
-              rb = which == 0 ? stg.q(j) : stg.k(e);
-              dst = (which == 0 ? KQ : KK) + j * 32 + l;
-            } else {
-              const int p = t - nout, ia = p / nf, jb = p - ia * nf;
-              if (jb >= ia) continue;
-              ra = stg.k(f0 + jb);
-              rb = stg.k(f0 + ia);
-              dst = Mf + ia * kMaxW + jb;
+        if (hf == 0 && (pre || post)) {
+          // ---- fold scalars (fold heads only): Gram dots k_i'.k_i in 4 x 4 blocks.
+          if (have) {
+            const int nb = (nf + 3) / 4;
+            for (int blk = gw; blk < nb * nb; blk += kGroupWarps) {
+              const int bi = blk / nb, bj = blk - bi * nb;
+              if (bj > bi) continue;
+              float part[16];
+              float4 ka[4], kb[4];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int ia = 4 * bi + c, ib = 4 * bj + c;
+                ka[c] = ia < nf ? ld4<Tin>(stg.k(f0 + ia) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                kb[c] = ib < nf ? ld4<Tin>(stg.k(f0 + ib) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+              for (int ca = 0; ca < 4; ++ca)
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) part[ca * 4 + cb] = dot4(ka[ca], kb[cb]);
+              tr_sum<16, 16>(part, lane);
+              const int idx = tr_base<16, 16>(lane);
+              const int ia = 4 * bi + idx / 4, ib = 4 * bj + idx % 4;
+              if ((lane & 1) == 0 && ib < ia && ia < nf) {
+                // A[i][i'] = beta_i e^{seg(i', i)} k_i'.k_i (direct sums)
+                float sgm = 0.0f;
+                for (int r = ib + 1; r <= ia; ++r) sgm += gw_[f0 + r];
+                Mf[ia * kMaxW + ib] = bw_[f0 + ia] * expf(sgm) * part[0];
+              }
             }
-            float acc = dot4(ld4<Tin>(ra + c0), ld4<Tin>(rb + c0));
-            acc = warp_sum(acc);
-            if (lane == 0) *dst = acc;
-          }
-          if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
-          // ---- decays: warp j < m handles output j; one warp the fold.
-          for (int task = gw; !failed && task < MAXM + 1; task += kGroupWarps) {
-            if (task < MAXM) {
-              if (task >= m) continue;
-              const int e = n + task, len = e - w0 + 1;
-              const float v = lane < len ? gw_[w0 + lane] : 0.0f;
-              float after, total;
-              suffix_scan(v, lane, after, total);
-              const float ex = expf(after);
-              Mq[task * 32 + lane] = lane < len ? ex * KQ[task * 32 + lane] : 0.0f;
-              Mk[task * 32 + lane] = lane < len - 1 ? ex * KK[task * 32 + lane] : 0.0f;
-              if (lane == 0) odec[task] = expf(total);
-            } else if (pre || post) {
+            if (gw == 1 % kGroupWarps) {   // fold weights
               const float v = lane < nf ? gw_[f0 + lane] : 0.0f;
               float after, total;
               suffix_scan(v, lane, after, total);
               fw[lane] = expf(after);
               if (lane == 0) decF[0] = expf(total);
-              // e^{G_i}: sum of g from the window start to entry i (direct sums)
-              float pre_sum = 0.0f;
+              float pre_sum = 0.0f;   // e^{G_i}: g summed from the window start to entry i
               for (int r = 0; r <= lane && r < nf; ++r) pre_sum += gw_[f0 + r];
               decf[lane] = expf(pre_sum);
               if (pre && post && lane == 0) {   // L = 1: then fold the new entry alone
                 one[0] = expf(gw_[n]);
                 one[1] = 1.0f;
+                one[2] = 1.0f;
               }
             }
           }
-          if (!failed && (pre || post)) {   // Mf[i][i'] *= e^{seg(i', i)}, direct sums
-            for (int p = gt; p < nf * nf; p += kGroupThreads) {
-              const int i = p / nf, ip = p - i * nf;
-              if (ip >= i) continue;
-              float sgm = 0.0f;
-              for (int r = ip + 1; r <= i; ++r) sgm += gw_[f0 + r];
-              Mf[i * kMaxW + ip] *= expf(sgm);
+          if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
+          if (!failed && gw == 0) {
+            // T = (I + A)^{-1}: unit lower triangular, lane c computes column c
+            // by forward substitution (it reads only its own column of T).
+            const int c = lane;
+            for (int i = 0; i < nf; ++i) {
+              float v = i == c ? 1.0f : 0.0f;
+              if (i > c) {
+                float acc = 0.0f;
+                for (int ip = c; ip < i; ++ip) acc = fmaf(Mf[i * kMaxW + ip], Tm[ip * kMaxW + c], acc);
+                v = -acc;
+              }
+              if (c < nf) Tm[i * kMaxW + c] = v;
             }
           }
           if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
@@ -506,7 +596,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             for (int r = 0; r < RPW; ++r)
               f[r] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(urow0 + r) * DK + c0) * 4);
           }
-          fold_rows<Tin>(f, stg, f0, nf, decf, Mf, fw, decF[0], bw_, urow0, U, lane, c0);
+          fold_rows<Tin>(f, stg, f0, nf, decf, Tm, fw, decF[0], bw_, urow0, U, lane, c0);
 #pragma unroll
           for (int r = 0; r < RPW; ++r) {
             const int row = urow0 + r;
@@ -570,6 +660,17 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           const int base = tr_base<NV, 16>(lane);
           constexpr int R = NV >= 32 ? NV / 32 : 1;
           constexpr int DUP = NV >= 32 ? 1 : 32 / NV;
+          if constexpr (MAXM == 1) {
+            // one token: the lane holds z or a of its row; the other sits in lane ^ 2
+            const float other = __shfl_xor_sync(kFull, part[0], 2);
+            const int r = base >> 1, which = base & 1, row = urow0 + r, e = n;
+            const float z = which == 0 ? part[0] : other, av = which == 0 ? other : part[0];
+            const float wv = bw_[e] * (to_f32<Tin>(stg.v(e)[row]) - z);
+            if ((lane & 1) == 0) {
+              if (which == 0) wring[((bh * 2 + hf) * cap + (st + e) % cap) * HALF + row] = wv;
+              else a.out[((size_t)b * a.H + h) * DV + hf * HALF + row] = a.out_scale * fmaf(Mq[e - w0], wv, av);
+            }
+          } else {
           if ((lane & (DUP - 1)) == 0) {
 #pragma unroll
             for (int q = 0; q < R; ++q) red[base + q] = part[q];
@@ -590,6 +691,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             }
           }
           __syncwarp();
+          }
         }
 
         if (post) {   // the decode filled the window: fold all of it (from fp32)
@@ -598,9 +700,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             for (int r = 0; r < RPW; ++r) f[r] = vw[r];
           }
           if (pre)   // L = 1: the window is the new entry alone
-            fold_rows<Tin>(f, stg, n, 1, one, Mf, one + 1, one[0], bw_, urow0, U, lane, c0);
+            fold_rows<Tin>(f, stg, n, 1, one, one + 2, one + 1, one[0], bw_, urow0, U, lane, c0);
           else
-            fold_rows<Tin>(f, stg, f0, nf, decf, Mf, fw, decF[0], bw_, urow0, U, lane, c0);
+            fold_rows<Tin>(f, stg, f0, nf, decf, Tm, fw, decF[0], bw_, urow0, U, lane, c0);
 #pragma unroll
           for (int r = 0; r < RPW; ++r) {
             const int row = urow0 + r;
@@ -706,22 +808,28 @@ template <typename Tin, int RF, int MAXM>
 cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
   using HS = HeadScalars<MAXM>;
   auto kern = gdn_replay_kernel<Tin, RF, MAXM>;
-  int hc = a.H < 16 ? a.H : 16;
-  while (a.H % hc) --hc;
   const size_t esz = sizeof(Tin);
   const size_t krow = DK * esz, vhrow = HALF * esz;
   const size_t stage = ((size_t)tile_bytes<RF>() + scale_bytes<RF>() + (a.L + MAXM) * krow + MAXM * krow +
                         (a.L + MAXM) * vhrow + (size_t)a.L * HALF * 4 + 127) & ~(size_t)127;
   const size_t wmax = a.L + MAXM;
-  const size_t group_floats = (2 * hc * wmax + HS::kOut + HS::kFold + HS::kDots + kGroupWarps * HS::kWarp + 31) & ~(size_t)31;
-  const size_t fixed = kGroups * sizeof(float) * group_floats;
   int dev = 0, sms = 0, max_smem = 0;
   cudaError_t e;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   const size_t budget = (size_t)max_smem - 2048;
-  if (fixed + 2 * stage > budget) return cudaErrorInvalidConfiguration;
+  // heads per item: the largest divisor of H (at most 16) whose per-head scalars
+  // leave room for at least two stages
+  int hc = a.H < 16 ? a.H : 16;
+  size_t fixed = 0;
+  for (;; --hc) {
+    if (hc < 1) return cudaErrorInvalidConfiguration;
+    if (a.H % hc) continue;
+    const size_t group_floats = (2 * hc * wmax + (size_t)hc * HS::kOut + HS::kFold + kGroupWarps * HS::kWarp + 31) & ~(size_t)31;
+    fixed = kGroups * sizeof(float) * group_floats;
+    if (fixed + 2 * stage <= budget) break;
+  }
   int stages = (int)((budget - fixed) / stage);
   if (stages > kMaxStages) stages = kMaxStages;
   const size_t smem = fixed + (size_t)stages * stage;
