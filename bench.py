@@ -46,7 +46,10 @@ POOL = 32
 
 
 # ------------------------------------------------------------------ helpers
-def dist_setup(ngpus):
+def dist_setup(ngpus, backend="nccl"):
+    """One process per GPU (torch.distributed.run sets RANK / LOCAL_RANK /
+    WORLD_SIZE).  Replicas only: the process group carries the start/stop
+    barriers and the max-over-ranks of the timings, never decode data."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -54,10 +57,18 @@ def dist_setup(ngpus):
         raise SystemExit(f"--gpus {ngpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return rank, world, local
+
+
+def job_throughput(world, tokens_per_step, steps, elapsed_max):
+    """Whole-job tokens/s: every rank decodes its own batch; the slowest rank's
+    device time bounds the job."""
+    return world * tokens_per_step * steps / elapsed_max
 
 
 def barrier(world):
@@ -172,17 +183,21 @@ class Mamba2Work:
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
 
-    def __init__(self, dev, seed, batch=None):
-        from hybrid_ssm_decode_replayssm_b200 import rssm
-        self.shape = s = si.MAMBA2_SERVING if batch is None else si.MAMBA2_SERVING.with_(batch=batch)
+    def __init__(self, dev, seed, batch=None, read_fmt=0, window=None):
+        self.shape = s = (si.MAMBA2_SERVING if batch is None else si.MAMBA2_SERVING.with_(batch=batch))
+        if window is not None:
+            self.shape = s = s.with_(window=window, max_draft=min(s.max_draft, window))
+        self.seed, self.dev, self.read_fmt = seed, dev, read_fmt
         A, D = si.mamba2_params(s, seed)
         self.A, self.D = A.to(dev), D.to(dev)
         self.h0 = si.mamba2_checkpoint(s, seed).to(dev)
-        self.desc = rssm.make_desc(rssm.RSSM_MAMBA2, s.batch, s.nheads, s.headdim, s.dstate,
-                                   ngroups=s.ngroups, window=s.window, max_draft=s.max_draft,
-                                   in_dtype=rssm.RSSM_BF16)
         self.host_pool = [si.mamba2_tokens(s, t, seed) for t in range(POOL)]
         self.pool = [[tok[k].to(dev) for k in self.keys] for tok in self.host_pool]
+        if dev.type == "cuda":
+            from hybrid_ssm_decode_replayssm_b200 import rssm
+            self.desc = rssm.make_desc(rssm.RSSM_MAMBA2, s.batch, s.nheads, s.headdim, s.dstate,
+                                       ngroups=s.ngroups, window=s.window, max_draft=s.max_draft,
+                                       in_dtype=rssm.RSSM_BF16, read_fmt=read_fmt)
         self.out_shape = (s.batch, s.nheads, s.headdim)
         self.tokens_per_call = s.batch
         self.workload = (f"Mamba-2 decode layer: batch {s.batch}, {s.nheads} heads, headdim {s.headdim}, "
@@ -191,6 +206,9 @@ class Mamba2Work:
     def layer(self):
         from hybrid_ssm_decode_replayssm_b200 import rssm
         return rssm.ReplayLayer(self.desc, self.h0.clone(), self.A, self.D)
+
+    def drafts(self, rnd, k):
+        return [t.to(self.dev) for t in (si.mamba2_drafts(self.shape, rnd, k, self.seed)[n] for n in self.keys)]
 
     def bytes_per_call(self, pos):
         """Algorithmic bytes of the decode call at window position pos (1..L)."""
@@ -228,14 +246,18 @@ class GDNWork:
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
 
-    def __init__(self, dev, seed, batch=None):
-        from hybrid_ssm_decode_replayssm_b200 import rssm
+    def __init__(self, dev, seed, batch=None, read_fmt=0, window=None):
         self.shape = s = si.GDN_SERVING if batch is None else si.GDN_SERVING.with_(batch=batch)
+        if window is not None:
+            self.shape = s = s.with_(window=window, max_draft=min(s.max_draft, window))
+        self.seed, self.dev, self.read_fmt = seed, dev, read_fmt
         self.h0 = si.gdn_checkpoint(s, seed).to(dev)
-        self.desc = rssm.make_desc(rssm.RSSM_GDN, s.batch, s.nheads, s.dv, s.dk, window=s.window,
-                                   max_draft=s.max_draft, in_dtype=rssm.RSSM_BF16)
         self.host_pool = [si.gdn_tokens(s, t, seed) for t in range(POOL)]
         self.pool = [[tok[k].to(dev) for k in self.keys] for tok in self.host_pool]
+        if dev.type == "cuda":
+            from hybrid_ssm_decode_replayssm_b200 import rssm
+            self.desc = rssm.make_desc(rssm.RSSM_GDN, s.batch, s.nheads, s.dv, s.dk, window=s.window,
+                                       max_draft=s.max_draft, in_dtype=rssm.RSSM_BF16, read_fmt=read_fmt)
         self.out_shape = (s.batch, s.nheads, s.dv)
         self.tokens_per_call = s.batch
         self.workload = (f"Gated DeltaNet decode layer: batch {s.batch}, {s.nheads} heads, d_k = d_v = {s.dk}, "
@@ -244,6 +266,9 @@ class GDNWork:
     def layer(self):
         from hybrid_ssm_decode_replayssm_b200 import rssm
         return rssm.ReplayLayer(self.desc, self.h0.clone())
+
+    def drafts(self, rnd, k):
+        return [t.to(self.dev) for t in (si.gdn_drafts(self.shape, rnd, k, self.seed)[n] for n in self.keys)]
 
     def bytes_per_call(self, pos):
         """Algorithmic bytes of the decode call at window position pos (1..L)."""
@@ -401,6 +426,107 @@ def cpu_baseline(work, seed, budget_s=12.0):
             "seconds": round(el, 2)}
 
 
+def time_plain_decode(work, layer, steps, warmup, L):
+    """Device time of `steps` windows of L decode calls (no per-launch events)."""
+    out = torch.empty(work.out_shape, device=work.dev)
+    t = 0
+    for _ in range(warmup * L):
+        layer.decode_step(work.pool[t % POOL], out)
+        t += 1
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps * L):
+        layer.decode_step(work.pool[t % POOL], out)
+        t += 1
+    stop.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop) / 1e3
+
+
+def speculative_leg(work, rounds=48, warmup=4, k=4):
+    """Verify k drafts, accept a seeded prefix U{0..k} per sequence, roll back the
+    rest (a fold happens inside verify when the window cannot take k more).
+    Baseline: snapshot verify, k conventional steps each writing a new state copy."""
+    B = work.shape.batch
+    layer = work.layer()
+    drafts = [work.drafts(r, k) for r in range(8)]
+    accepts = [si.accept_counts(B, r, k, work.seed) for r in range(rounds + warmup)]
+    rejects = [(k - a).to(torch.int32).to(work.dev) for a in accepts]
+    out = torch.empty((B, k) + work.out_shape[1:], device=work.dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for r in range(warmup):
+        layer.verify(k, drafts[r % 8], out)
+        layer.rollback(rejects[r])
+    e0, e1 = ev(), ev()
+    rb = [(ev(), ev()) for _ in range(rounds)]
+    torch.cuda.synchronize()
+    e0.record()
+    for r in range(rounds):
+        layer.verify(k, drafts[r % 8], out)
+        rb[r][0].record()
+        layer.rollback(rejects[warmup + r])
+        rb[r][1].record()
+    e1.record()
+    torch.cuda.synchronize()
+    el = e0.elapsed_time(e1) / 1e3
+    rollback_us = statistics.mean(a.elapsed_time(b) for a, b in rb) * 1e3
+    accepted = sum(int(a.sum()) for a in accepts[warmup:])
+    status = layer.get_status()
+    del layer
+    # snapshot baseline: k snapshots of the full state per round
+    snaps = [work.h0.clone() for _ in range(k + 1)]
+    base = work.layer()
+    one = torch.empty(work.out_shape, device=work.dev)
+    draft_tokens = [[[t[:, j].contiguous() for t in drafts[r]] for j in range(k)] for r in range(8)]
+    def snapshot_round(r):
+        for j in range(k):
+            base.conventional_step(snaps[j], snaps[j + 1], draft_tokens[r % 8][j], one)
+    for r in range(warmup):
+        snapshot_round(r)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for r in range(rounds):
+        snapshot_round(r)
+    e1.record()
+    torch.cuda.synchronize()
+    el_base = e0.elapsed_time(e1) / 1e3
+    del base, snaps
+    return {"k": k, "rounds": rounds, "verified_tokens_per_s": round(B * k * rounds / el, 1),
+            "accepted_tokens_per_s": round(accepted / el, 1),
+            "round_us": round(el / rounds * 1e6, 2), "rollback_us": round(rollback_us, 2),
+            "mean_accepted": round(accepted / (B * rounds), 3), "status_bits": status,
+            "snapshot_baseline": {"round_us": round(el_base / rounds * 1e6, 2),
+                                  "accepted_tokens_per_s": round(accepted / el_base, 1),
+                                  "how": f"{k} conventional steps per round, each writing a new full-state snapshot"},
+            "speedup_vs_snapshot": round(el_base / el, 3)}
+
+
+def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6):
+    """Replay decode tokens/s with the fp32 checkpoint read directly and with an
+    FP8 / NVFP4 read copy, per window length (checkpoint and tokens of `base`)."""
+    import copy
+    from hybrid_ssm_decode_replayssm_b200 import rssm
+    res = {}
+    for name, fmt in (("fp32", rssm.RSSM_READ_FP32), ("fp8_e4m3_row", rssm.RSSM_READ_FP8_E4M3_ROW),
+                      ("nvfp4", rssm.RSSM_READ_NVFP4)):
+        row = {}
+        for L in windows:
+            work = copy.copy(base)
+            work.shape = base.shape.with_(window=L, max_draft=min(base.shape.max_draft, L))
+            work.desc = copy.copy(base.desc)
+            work.desc.window, work.desc.max_draft, work.desc.read_fmt = L, min(base.shape.max_draft, L), fmt
+            layer = work.layer()
+            n_windows = max(2, (steps * 16) // L)
+            el = time_plain_decode(work, layer, n_windows, 2, L)
+            row[f"L{L}"] = round(work.shape.batch * L * n_windows / el, 1)
+            del layer
+            torch.cuda.empty_cache()
+        res[name] = row
+    return res
+
+
 # -------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -413,7 +539,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
-    ap.add_argument("--legs", default="replay,conventional,e2e",
+    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -423,8 +549,11 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     seed = args.seed + rank
-    work = WORKLOADS[args.layer](dev, seed, args.batch)
     legs = set(args.legs.split(","))
+    if args.impl == "reference":   # the oracle runs on the host: build the workload there
+        work = WORKLOADS[args.layer](torch.device("cpu"), seed, args.batch)
+    else:
+        work = WORKLOADS[args.layer](dev, seed, args.batch)
     L = work.shape.window
     tokens_per_step = work.tokens_per_call * L
     cfg = {"workload": work.workload, "global_batch": work.shape.batch * world,
@@ -453,7 +582,7 @@ def main():
     elapsed, per, positions, launches, clocks = time_replay(work, layer, args.steps, args.warmup, L,
                                                             out, dev, world, local)
     elapsed = max_over_ranks(elapsed, world, dev)
-    value = world * tokens_per_step * args.steps / elapsed
+    value = job_throughput(world, tokens_per_step, args.steps, elapsed)
 
     alg_bytes = sum(work.bytes_per_call(p) for p in positions)    # per-launch pass
     kern_time = sum(per)
@@ -488,6 +617,41 @@ def main():
                "how": "rssm_decode_step per call with pinned-host inputs copied in and outputs "
                       "copied out, pipelined on copy streams"}
 
+    extras = {}
+    if "e2e" in legs:
+        del e2e_layer
+    gw = None
+    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy"}:
+        gw = GDNWork(dev, seed, args.batch)
+    if world == 1 and "gdn" in legs and gw is not None:
+        gl = gw.layer()
+        gout = torch.empty(gw.out_shape, device=dev)
+        g_el, g_per, g_pos, _, _ = time_replay(gw, gl, max(20, args.steps // 3), args.warmup, L, gout, dev, 1, local)
+        g_steps = max(20, args.steps // 3)
+        g_bytes = sum(gw.bytes_per_call(p) for p in g_pos)
+        gc_el = time_conventional(gw, gl, g_steps, args.warmup, L, gout, 1)
+        extras["gdn"] = {"workload": gw.workload, "value": round(gw.tokens_per_call * L * g_steps / g_el, 1),
+                         "unit": "tokens/s", "hbm_gbs": round(g_bytes / g_el / 1e9, 1),
+                         "roofline_frac": round(g_bytes / sum(g_per) / 1e9 / measured_peak()[0], 4),
+                         "launch_us_fold": round(statistics.mean(p for p, q in zip(g_per, g_pos) if q == L) * 1e6, 2),
+                         "launch_us_nofold": round(statistics.mean(p for p, q in zip(g_per, g_pos) if q != L) * 1e6, 2),
+                         "conventional_tokens_per_s": round(gw.tokens_per_call * L * g_steps / gc_el, 1),
+                         "replay_speedup": round(gc_el / g_el, 3)}
+        del gl
+        torch.cuda.empty_cache()
+    if world == 1 and "speculative" in legs:
+        extras["speculative"] = {"mamba2": speculative_leg(work)}
+        torch.cuda.empty_cache()
+        if gw is not None:
+            extras["speculative"]["gdn"] = speculative_leg(gw)
+            torch.cuda.empty_cache()
+    if world == 1 and "read_copy" in legs:
+        extras["read_copy"] = {work.name: read_copy_leg(work)}
+        if gw is not None:
+            extras["read_copy"]["gdn"] = read_copy_leg(gw)
+    del gw
+    torch.cuda.empty_cache()
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(work, seed)
@@ -500,7 +664,7 @@ def main():
                 "data": "synthetic (seeded; bf16 inputs, fp32 checkpoint)", "config": cfg,
                 "hbm_gbs": round(alg_bytes / elapsed / 1e9 * world, 1),   # same calls, headline pass
                 "roofline": roofline, "clocks": clocks, "gpu_launches": int(launches),
-                "e2e": e2e, "conventional": conv,
+                "e2e": e2e, "conventional": conv, **extras,
                 "cpu_baseline": cb}
         print(json.dumps(line), flush=True)
     if world > 1:
