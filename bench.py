@@ -412,13 +412,13 @@ def time_e2e(work, layer, steps, warmup, L, dev, world):
     return start.elapsed_time(stop) / 1e3, in_bytes * L, out_bytes * L
 
 
-def cpu_baseline(work, seed, budget_s=12.0):
-    """The fp64 oracle as it stands, single-threaded (BLAS pinned to 1 thread)."""
+def cpu_baseline(work, seed, budget_s=12.0, nseq=16):
+    """The fp64 oracle as it stands, single-threaded (BLAS pinned to 1 thread), on
+    `nseq` sequences for about `budget_s` seconds."""
     from threadpoolctl import threadpool_limits
-    nseq = 8
     with threadpool_limits(1):
-        t1 = work.oracle_sample(nseq, 1, seed)
-        steps = max(2, min(64, int(budget_s / max(t1, 1e-3))))
+        t1 = work.oracle_sample(nseq, 2, seed) / 2
+        steps = max(2, min(1024, int(budget_s / max(t1, 1e-4))))
         el = work.oracle_sample(nseq, steps, seed)
     return {"value": nseq * steps / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": (f"{nseq} of {work.shape.batch} sequences (all {work.shape.nheads} heads), "

@@ -16,15 +16,22 @@
 // paragraphs 2-4): outputs come from the checkpoint and the buffered inputs,
 // the buffer is folded in when it fills, drafts are appended and rolled back
 // by pointer, and a low-precision copy may serve the reads while the
-// recurrence stays in high precision.  So a fold never uses the cached w: it
-// solves the window again from the fp32 checkpoint.
+// recurrence stays in high precision.  A layer that reads the fp32 checkpoint
+// solved its cached w against that checkpoint, so its fold is the rank-l
+// update with them; a layer that reads a low-precision copy solved its cached
+// w against the copy, so its fold solves the window again from the fp32
+// checkpoint (UT transform) and the copy's rounding never enters the state.
 //
 // Work unit: half a head (64 of the 128 value rows, 32 KiB of fp32 state).  A
 // persistent CTA has one producer warp, which streams units into a ring of
-// shared-memory stages with 1-D TMA bulk copies, and two consumer groups of 8
-// warps taking alternate items (item = one sequence and a chunk of heads).
-// Per head the group first computes the head's scalars (k.k and k.q products
-// and decays) from the stage, then each warp handles 8 rows of each half.
+// shared-memory stages with 1-D TMA bulk copies (the read tile and the cached
+// w rows; fold units also the window's k and v rows), and two consumer groups
+// of 8 warps taking alternate items (item = one sequence and a chunk of
+// heads), whose units the producer interleaves (IssueOrder).  An item's
+// prologue converts the new q, k, v rows to fp32 in shared memory, appends k
+// and v to the ring and computes every head's window scalars.  Per unit each warp owns 8 state rows; a row is spread over 8
+// lanes (4 chunks of 4 columns each), so its dot products reduce in three
+// shuffle steps.
 #include "rssm_device.cuh"
 
 namespace rssm {
@@ -38,7 +45,7 @@ constexpr int kConsumers = kGroups * kGroupThreads;
 constexpr int kReplayThreads = kConsumers + 32;
 constexpr int kMaxStages = 16;
 constexpr int RPW = HALF / kGroupWarps;   // rows of a unit per warp (8)
-constexpr int kMaxW = 32;                 // longest window a scan or fold covers
+constexpr int kMaxW = 32;                 // window positions a scalar array covers
 
 template <int RF> constexpr int tile_bytes() {
   return RF == RSSM_READ_FP32 ? HALF * DK * 4 : RF == RSSM_READ_FP8_E4M3_ROW ? HALF * DK : HALF * DK / 2;
@@ -59,18 +66,6 @@ __device__ __forceinline__ float4 ld4(const Tin *p) {
     return make_float4(to_f32<Tin>(e[0]), to_f32<Tin>(e[1]), to_f32<Tin>(e[2]), to_f32<Tin>(e[3]));
   }
 }
-template <typename Tin>
-__device__ __forceinline__ void ld8(const Tin *p, float (&o)[8]) {
-  if constexpr (sizeof(Tin) == 4) {
-    const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
-    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-  } else {
-    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
-    const Tin *e = reinterpret_cast<const Tin *>(&raw);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = to_f32<Tin>(e[q]);
-  }
-}
 __device__ __forceinline__ float dot4(const float4 a, const float4 b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
@@ -79,26 +74,39 @@ __device__ __forceinline__ void fma4(float4 &t, float c, const float4 k) {
 }
 __device__ __forceinline__ void scale4(float4 &t, float c) { t.x *= c; t.y *= c; t.z *= c; t.w *= c; }
 
-// Stage layout of one unit: [read tile | scales | k rows | q rows | v half rows | w half rows].
-// k and v rows: committed entries at rows [0, n), new tokens at rows L + j.
-template <typename Tin>
-struct GStage {
-  uint8_t *base;
-  int koff, qoff, voff, woff, n, L;
-  __device__ __forceinline__ int slot_row(int i) const { return i < n ? i : L + (i - n); }
-  __device__ __forceinline__ const Tin *k(int i) const {
-    return reinterpret_cast<const Tin *>(base + koff) + (size_t)slot_row(i) * DK;
-  }
-  __device__ __forceinline__ const Tin *q(int j) const {
-    return reinterpret_cast<const Tin *>(base + qoff) + (size_t)j * DK;
-  }
-  __device__ __forceinline__ const Tin *v(int i) const {
-    return reinterpret_cast<const Tin *>(base + voff) + (size_t)slot_row(i) * HALF;
-  }
-  __device__ __forceinline__ const float *w(int i) const {
-    return reinterpret_cast<const float *>(base + woff) + (size_t)i * HALF;
-  }
+// Shared-memory layout of a replay launch (the host sizes the launch with the
+// same function).  Stage, in bytes: [read tile | scales | cached w rows (L) |
+// k rows (L + MAXM, fold units) | v half rows (L + MAXM, fold units of
+// re-solving layers)]; committed entries at rows [0, n), new tokens at L + j.
+// Group region, in floats: gates and betas of the item's heads, fp32 k/q/v of
+// the new tokens, per-head output scalars, fold scalars, per-warp scratch.
+struct Layout {
+  int woff, koff, voff, stage_bytes;
+  int sg, sbeta, kqv, hso, fold, warp, warp_floats, group_floats;
 };
+template <typename Tin, int RF, int MAXM>
+__host__ __device__ inline Layout make_layout(int L, int hc) {
+  constexpr bool kResolve = RF != RSSM_READ_FP32;
+  Layout y;
+  const int krow = DK * (int)sizeof(Tin), vhrow = HALF * (int)sizeof(Tin);
+  y.woff = tile_bytes<RF>() + scale_bytes<RF>();
+  y.koff = y.woff + L * HALF * 4;
+  y.voff = y.koff + (L + MAXM) * krow;
+  y.stage_bytes = (y.voff + (kResolve ? (L + MAXM) * vhrow : 0) + 127) & ~127;
+  const int wmax = L + MAXM;
+  y.sg = 0;
+  y.sbeta = hc * wmax;
+  y.kqv = (2 * hc * wmax + 3) & ~3;
+  y.hso = y.kqv + hc * 3 * MAXM * DK;
+  y.fold = y.hso + hc * (MAXM + 2 * MAXM * kMaxW);
+  // fw[2][kMaxW + 1] | decF[2] | decf[2][kMaxW + 1] | A[L][L] | T[L][L] (A, T: re-solving layers)
+  const int fold_floats = 4 * (kMaxW + 1) + 2 + (kResolve ? 2 * L * L : 0);
+  y.warp = (y.fold + fold_floats + 3) & ~3;
+  // per warp: red[8][MAXM][2] | win[8][MAXM][2] | wnew[MAXM][8] | U[L][8] (re-solving layers)
+  y.warp_floats = (5 * MAXM * RPW + (kResolve ? L * RPW : 0) + 3) & ~3;
+  y.group_floats = (y.warp + kGroupWarps * y.warp_floats + 31) & ~31;
+  return y;
+}
 
 struct RowPlan {
   int st, n;
@@ -131,80 +139,54 @@ __device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
   return r;
 }
 
-// Per-group shared scalars of the current head.
-template <int MAXM>
-struct HeadScalars {
-  static constexpr int kOut = MAXM + 2 * MAXM * 32;             // per head: dec, Mk, Mq
-  static constexpr int kFold = kMaxW + 2 * kMaxW * kMaxW + kMaxW + 4; // decf, A, T, fw, decF, 1-entry fold
-  static constexpr int kDots = 0;
-  static constexpr int kWarp = kMaxW * RPW + 2 * MAXM * RPW;     // U/W fold scratch, reductions
-};
-
-// Fold of the window entries [i0, i0 + nf) into the fp32 rows t (8 rows of this
-// warp, 4 columns of this lane), by the UT transform of the window: with
-// u_i = t k_i (matvecs in chunks of 4 keys), r_i = beta_i (v_i - e^{G_i} u_i)
-// and T = (I + A)^{-1}, A[i][i'] = beta_i e^{seg(i',i)} k_i'.k_i (i' < i), the
-// solved values are w = T r (forward substitution done once per head in T),
-// then t <- decF t + sum_i fw_i w_i k_i^T.
-template <typename Tin>
-__device__ void fold_rows(float4 (&t)[RPW], const GStage<Tin> &stg, int i0, int nf, const float *decf,
-                          const float *Tm, const float *fw, float decF, const float *beta, int urow0,
-                          float *U, int lane, int c0) {
-  for (int ch = 0; ch < nf; ch += 4) {
-    float part[RPW * 4];
+// Quantise two state rows held in the 8-lane row mapping (lane j of the row's
+// lane group holds columns 32 c + 4 j .. + 3, c = 0..3) into the read copy,
+// returning the dequantised values.  FP8: one fp32 scale per row; NVFP4: one
+// E4M3 scale per 16 columns (4 lanes of one chunk).
+template <int RF>
+__device__ __forceinline__ void quantize_rows(const float4 (&x)[2][4], float4 (&out)[2][4], uint8_t *rc,
+                                              void *scales, size_t row_base, int row_a, int row_b, int j,
+                                              int lane) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = ch + c;
-      const float4 kc = i < nf ? ld4<Tin>(stg.k(i0 + i) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < 2; ++r) {
+    const int row = r == 0 ? row_a : row_b;
+    uint8_t *crow = rc + (size_t)row * rc_row_bytes<RF>();
+    if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+      float am = 0.0f;
 #pragma unroll
-      for (int r = 0; r < RPW; ++r) part[r * 4 + c] = dot4(t[r], kc);
+      for (int c = 0; c < 4; ++c)
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(x[r][c].x), fabsf(x[r][c].y)), fmaxf(fabsf(x[r][c].z), fabsf(x[r][c].w))));
+      am = group_max<8>(am);
+      const float s = am / 448.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w = 0;
+        if (s != 0.0f)
+          w = enc_e4m3(x[r][c].x / s) | (enc_e4m3(x[r][c].y / s) << 8) | (enc_e4m3(x[r][c].z / s) << 16) |
+              (enc_e4m3(x[r][c].w / s) << 24);
+        *reinterpret_cast<uint32_t *>(crow + 32 * c + 4 * j) = w;
+        dec_e4m3x4(w, s, out[r][c]);
+      }
+      if (j == 0) reinterpret_cast<float *>(scales)[row_base + row] = s;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        out[r][c] = quantize4<RSSM_READ_NVFP4, 8>(x[r][c], crow, scales, row_base + row, DK, 32 * c + 4 * j, lane);
     }
-    tr_sum<RPW * 4, 16>(part, lane);
-    const int idx = tr_base<RPW * 4, 16>(lane), r = idx / 4, i = ch + idx % 4;
-    if (i < nf) U[i * RPW + r] = part[0];
   }
-  __syncwarp();
-  for (int p = lane; p < nf * RPW; p += 32) {   // r_i per (entry, row); U[i][r] layout
-    const int i = p / RPW, r = p - i * RPW;
-    U[p] = beta[i0 + i] * fmaf(-decf[i], U[p], to_f32<Tin>(stg.v(i0 + i)[urow0 + r]));
-  }
-  __syncwarp();
-  constexpr int kPer = kMaxW * RPW / 32;
-  float wv[kPer];
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int p = lane + 32 * q, i = p / RPW, r = p - i * RPW;
-    float acc = 0.0f;
-    if (i < nf)
-      for (int ip = 0; ip <= i; ++ip) acc = fmaf(Tm[i * kMaxW + ip], U[ip * RPW + r], acc);
-    wv[q] = acc;
-  }
-  __syncwarp();
-#pragma unroll
-  for (int q = 0; q < kPer; ++q)
-    if (lane + 32 * q < nf * RPW) U[lane + 32 * q] = wv[q];
-  __syncwarp();
-#pragma unroll
-  for (int r = 0; r < RPW; ++r) scale4(t[r], decF);
-  for (int i = 0; i < nf; ++i) {
-    const float4 kc = ld4<Tin>(stg.k(i0 + i) + c0);
-    const float f = fw[i];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) fma4(t[r], f * U[i * RPW + r], kc);
-  }
-  __syncwarp();
 }
 
 template <typename Tin, int RF, int MAXM>
 __global__ void __launch_bounds__(kReplayThreads, 1)
     gdn_replay_kernel(const StepArgs a, const int hc, const int stages) {
-  using HS = HeadScalars<MAXM>;
+  constexpr bool kResolve = RF != RSSM_READ_FP32;
   constexpr int KROW = DK * (int)sizeof(Tin);
   constexpr int VHROW = HALF * (int)sizeof(Tin);
   constexpr int TB = tile_bytes<RF>();
   constexpr int SB = scale_bytes<RF>();
   constexpr int RB = rc_row_bytes<RF>();
   constexpr int SR = rc_scale_row_bytes<RF>();
+  constexpr int HSO = MAXM + 2 * MAXM * kMaxW;   // per head: dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ int stage_use[kMaxStages];   // see the Mamba-2 kernel: gates parity waits
@@ -212,16 +194,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L, cap = a.cap, m = a.m, WMAX = L + MAXM;
+  const Layout Y = make_layout<Tin, RF, MAXM>(L, hc);
   const int nchunk = a.H / hc;
   const int nitems = a.B * nchunk;
   const int my_items = (int)blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int total_seq = my_items * hc * 2;
-  const int KOFF = TB + SB;
-  const int QOFF = KOFF + (L + MAXM) * KROW;
-  const int VOFF = QOFF + MAXM * KROW;
-  const int WOFF = VOFF + (L + MAXM) * VHROW;
-  const size_t stage_bytes = ((size_t)WOFF + (size_t)L * HALF * 4 + 127) & ~(size_t)127;
-  const int group_floats = (2 * hc * WMAX + hc * HS::kOut + HS::kFold + kGroupWarps * HS::kWarp + 31) & ~31;
 
   const Tin *qin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *kin = reinterpret_cast<const Tin *>(a.in[1]);
@@ -253,29 +230,34 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    // Issue order: the units of items 2p and 2p+1 interleaved (unit u of 2p, unit
-    // u of 2p+1, unit u+1 of 2p, ...), so both consumer groups work at once.
-    int b2[2] = {0, 0}, chunk2[2] = {0, 0}, s = 0, u = 0, cur_pair = -1;
-    RowPlan rp2[2] = {};
+    // Issue order: the units of items 2p and 2p + 1 alternate (see IssueOrder).
+    const IssueOrder<true> order(my_items, 2 * hc);
+    // the current item of each group (scalars, not arrays: no local memory)
+    int b_0 = 0, b_1 = 0, chunk_0 = 0, chunk_1 = 0, cur_0 = -1, cur_1 = -1;
+    RowPlan rp_0{}, rp_1{};
+    int s = 0, u = 0;
     int issued = 0;
     for (int seq = 0; seq < total_seq; ++seq) {
       if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
         atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
         break;
       }
-      const int p = seq / (4 * hc), within = seq - p * 4 * hc;
-      const bool paired = 2 * p + 1 < my_items;
-      const int gsel = paired ? (within & 1) : 0;
-      const int unit = paired ? (within >> 1) : within;
-      if (p != cur_pair) {
-        cur_pair = p;
-        for (int g2 = 0; g2 < (paired ? 2 : 1); ++g2) {
-          item_of(2 * p + g2, b2[g2], chunk2[g2]);
-          rp2[g2] = plan_row(a, b2[g2]);
+      int kc, unit;
+      order.unit_at(seq, kc, unit);
+      if (kc & 1) {
+        if (kc != cur_1) {
+          cur_1 = kc;
+          item_of(kc, b_1, chunk_1);
+          rp_1 = plan_row(a, b_1);
         }
+      } else if (kc != cur_0) {
+        cur_0 = kc;
+        item_of(kc, b_0, chunk_0);
+        rp_0 = plan_row(a, b_0);
       }
-      const int b = b2[gsel], chunk = chunk2[gsel];
-      const RowPlan &rp = rp2[gsel];
+      const bool g1 = kc & 1;
+      const int b = g1 ? b_1 : b_0, chunk = g1 ? chunk_1 : chunk_0;
+      const RowPlan rp = g1 ? rp_1 : rp_0;
       issued = seq + 1;
       if (rp.refuse) {
         mbar_arrive(&full[s]);
@@ -284,11 +266,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         const int h = chunk * hc + jh;
         const size_t bh = (size_t)b * a.H + h;
         const bool fold = rp.pre || rp.post;
-        const int nk = fold ? rp.n : 0;                // committed k rows (fold passes)
-        const int nv = fold ? rp.n : 0;                // committed v rows
-        const int nw = rp.pre ? 0 : rp.n;              // committed w rows
-        uint8_t *dst = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + (nk + 2 * m) * KROW + (nv + m) * VHROW + nw * HALF * 4));
+        // cached w rows: the reads of the committed entries, and the folds of
+        // layers that fold with them
+        const int nw = (kResolve && rp.pre) ? 0 : rp.n;
+        const int nk = fold ? rp.n : 0;                       // k rows of fold units
+        const int nv = (kResolve && fold) ? rp.n : 0;         // v rows of re-solving folds
+        const int mk = fold ? m : 0, mv = (kResolve && fold) ? m : 0;
+        uint8_t *dst = smem + s * Y.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + nw * HALF * 4 + (nk + mk) * KROW + (nv + mv) * VHROW));
         if constexpr (RF == RSSM_READ_FP32) {
           bulk_g2s(dst, a.hc + (bh * DV + hf * HALF) * DK, TB, &full[s]);
         } else {
@@ -296,26 +281,26 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + (bh * DV + hf * HALF) * SR, SB, &full[s]);
         }
         const int c1 = rp.n < cap - rp.st ? rp.n : cap - rp.st;   // ring segment lengths
+        if (nw > 0) {
+          const float *src = wring + (bh * 2 + hf) * cap * HALF;
+          const int w1 = nw < c1 ? nw : c1;
+          bulk_g2s(dst + Y.woff, src + (size_t)rp.st * HALF, w1 * HALF * 4, &full[s]);
+          if (nw > w1) bulk_g2s(dst + Y.woff + w1 * HALF * 4, src, (nw - w1) * HALF * 4, &full[s]);
+        }
         if (nk > 0) {
           const Tin *src = kring + bh * cap * DK;
-          bulk_g2s(dst + KOFF, src + (size_t)rp.st * DK, c1 * KROW, &full[s]);
-          if (nk > c1) bulk_g2s(dst + KOFF + c1 * KROW, src, (nk - c1) * KROW, &full[s]);
+          bulk_g2s(dst + Y.koff, src + (size_t)rp.st * DK, c1 * KROW, &full[s]);
+          if (nk > c1) bulk_g2s(dst + Y.koff + c1 * KROW, src, (nk - c1) * KROW, &full[s]);
         }
         if (nv > 0) {
           const Tin *src = vring + (bh * 2 + hf) * cap * HALF;
-          bulk_g2s(dst + VOFF, src + (size_t)rp.st * HALF, c1 * VHROW, &full[s]);
-          if (nv > c1) bulk_g2s(dst + VOFF + c1 * VHROW, src, (nv - c1) * VHROW, &full[s]);
+          bulk_g2s(dst + Y.voff, src + (size_t)rp.st * HALF, c1 * VHROW, &full[s]);
+          if (nv > c1) bulk_g2s(dst + Y.voff + c1 * VHROW, src, (nv - c1) * VHROW, &full[s]);
         }
-        if (nw > 0) {
-          const float *src = wring + (bh * 2 + hf) * cap * HALF;
-          bulk_g2s(dst + WOFF, src + (size_t)rp.st * HALF, c1 * HALF * 4, &full[s]);
-          if (nw > c1) bulk_g2s(dst + WOFF + c1 * HALF * 4, src, (nw - c1) * HALF * 4, &full[s]);
-        }
-        for (int j = 0; j < m; ++j) {
+        for (int j = 0; j < mk; ++j) {
           const size_t tok = ((size_t)b * m + j) * a.H + h;
-          bulk_g2s(dst + KOFF + (L + j) * KROW, kin + tok * DK, KROW, &full[s]);
-          bulk_g2s(dst + QOFF + j * KROW, qin + tok * DK, KROW, &full[s]);
-          bulk_g2s(dst + VOFF + (L + j) * VHROW, vin + tok * DV + hf * HALF, VHROW, &full[s]);
+          bulk_g2s(dst + Y.koff + (L + j) * KROW, kin + tok * DK, KROW, &full[s]);
+          if (j < mv) bulk_g2s(dst + Y.voff + (L + j) * VHROW, vin + tok * DV + hf * HALF, VHROW, &full[s]);
         }
       }
       *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
@@ -334,20 +319,24 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   // -------------------------------------------------------------- consumers
   const int gi = warp / kGroupWarps, gw = warp % kGroupWarps, gt = tid - gi * kGroupThreads;
   const int bar_id = 1 + gi;
-  float *gbase = reinterpret_cast<float *>(smem + stages * stage_bytes) + gi * group_floats;
-  float *sg = gbase;                          // [hc][WMAX]  ln alpha
-  float *sbeta = sg + hc * WMAX;              // [hc][WMAX]
-  float *hso = sbeta + hc * WMAX;             // per head: dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
-  float *hsf = hso + hc * HS::kOut;           // decf[32] | A[32][32] | T[32][32] | fw[32] | decF | one[3]
-  float *wscr = hsf + HS::kFold + gw * HS::kWarp;
-  float *U = wscr, *red = wscr + kMaxW * RPW;
-  float *odec = hso, *Mk = hso + MAXM, *Mq = Mk + MAXM * 32;   // repointed per head
-  float *decf = hsf, *Mf = hsf + kMaxW, *Tm = Mf + kMaxW * kMaxW, *fw = Tm + kMaxW * kMaxW;
-  float *decF = fw + kMaxW;
-  float *one = decF + 1;   // window-full fold of a 1-entry window after a pre-fold (L = 1):
-                           // one[0] = e^{g} (its decf and decF), one[1] = 1 (fw), one[2] = 1 (T)
-  const int c0 = lane * 4;
-  const int urow0 = gw * RPW;   // first row of this warp inside a unit
+  float *G = reinterpret_cast<float *>(smem + stages * Y.stage_bytes) + gi * Y.group_floats;
+  float *sg = G + Y.sg;          // [hc][WMAX]  ln alpha of the window entries
+  float *sbeta = G + Y.sbeta;    // [hc][WMAX]
+  float *kqv = G + Y.kqv;        // [hc][k | q | v][MAXM][128]  new tokens, fp32
+  float *hso = G + Y.hso;        // [hc][HSO]
+  float *fw = G + Y.fold;        // [2][kMaxW + 1]  fold weights e^{seg(i, last)}: pre-fold, window-full fold
+  float *decF = fw + 2 * (kMaxW + 1);   // [2]  decay over each fold window
+  float *decf = decF + 2;        // [2][kMaxW + 1]  e^{G_i} within each fold window (re-solving layers)
+  float *Am = decf + 2 * (kMaxW + 1), *Tm = Am + L * L;   // re-solving layers
+  float *wscr = G + Y.warp + gw * Y.warp_floats;
+  float *red = wscr;                    // [8][MAXM][2]  reduced S.k_e and S.q per row
+  float *win = red + 2 * MAXM * RPW;    // [8][MAXM][2]  window sums per row
+  float *wnew = win + 2 * MAXM * RPW;   // [MAXM][8]     solved w of the new tokens
+  float *U = wnew + MAXM * RPW;         // [L][8]        re-solving folds
+  const int c0 = lane * 4;              // full-row mapping (scalars): 4 columns per lane
+  const int g8 = lane >> 3, j8 = lane & 7;   // state mapping: rows g8, g8 + 4 of the warp; lane j8 of the row
+  const int urow0 = gw * RPW;           // first row of this warp inside a unit
+  const int row_a = urow0 + g8, row_b = urow0 + g8 + 4;
 
   for (int k = gi; k < my_items; k += kGroups) {
     int b, chunk;
@@ -360,21 +349,28 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     if (rp.refuse && rp.bit && chunk == 0 && gt == 0) atomicOr(a.status, rp.bit);
     const int w0 = pre ? n : 0;
     const int ntot = n + m;
-    // fold window [f0, f0 + nf): the committed entries (pre) or the full window (post)
-    const int f0 = pre ? 0 : w0, nf = pre ? n : n - w0 + 1;
+    const int slot_n = (st + n) % cap;   // ring slot of the first new entry
 
     if (!rp.refuse) {
-      // ---- gates and betas of the item's heads; ring appends of new tokens
+      // Window scalars are computed in tasks (head jh, batch of CE window
+      // entries) spread over the group's warps.  (Loading a task's ring k rows
+      // before the first barrier was measured slower: the registers it holds
+      // across the barrier spill.)
+      constexpr int CE = MAXM == 1 ? 8 : 4;   // window entries per reduction
+      const int nbatch = m > 0 ? (ntot - w0 + CE - 1) / CE : 0;
+      const int ntask = hc * nbatch;
+      // ---- gates and betas of the item's heads; ring appends of the new gates
       for (int idx = gt; idx < hc * ntot; idx += kGroupThreads) {
         const int jh = idx / ntot, i = idx - jh * ntot;
         const size_t bh = bh0 + jh;
-        const int slot = (st + i) % cap;
         float g, be;
         if (i < n) {
+          const int slot = (st + i) % cap;
           g = gring[bh * cap + slot];
           be = bring[bh * cap + slot];
         } else {
           const size_t tok = ((size_t)b * m + (i - n)) * a.H + h0 + jh;
+          const int slot = (slot_n + (i - n)) % cap;
           g = logf(alin[tok]);
           be = bein[tok];
           gring[bh * cap + slot] = g;
@@ -383,95 +379,112 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         sg[jh * WMAX + i] = g;
         sbeta[jh * WMAX + i] = be;
       }
+      // ---- new tokens: k, q, v rows to fp32 in shared memory; k and v appended to the ring
       constexpr int kPer = 16 / sizeof(Tin);
-      for (int idx = gt; idx < hc * m * 2 * (DK / kPer); idx += kGroupThreads) {
-        const int per = 2 * (DK / kPer);
-        const int r = idx / per, c = (idx - r * per) * kPer;   // c in [0, 2*DK): k row then v row
-        const int jh = r / m, j = r - jh * m;
-        const size_t bh = bh0 + jh;
+      constexpr int kLoads = DK / kPer;   // 16-byte loads per row
+      for (int idx = gt; idx < hc * m * 3 * kLoads; idx += kGroupThreads) {
+        const int c = (idx % kLoads) * kPer;
+        int r = idx / kLoads;
+        const int which = r % 3;   // 0 k, 1 q, 2 v
+        r /= 3;
+        const int j = r % m, jh = r / m;
         const size_t tok = ((size_t)b * m + j) * a.H + h0 + jh;
-        const int slot = (st + n + j) % cap;
-        if (c < DK) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(kin + tok * DK + c));
+        const Tin *src = (which == 0 ? kin : which == 1 ? qin : vin) + tok * DK + c;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src));
+        const Tin *e = reinterpret_cast<const Tin *>(&raw);
+        float *dst = kqv + ((size_t)(jh * 3 + which) * MAXM + j) * DK + c;
+#pragma unroll
+        for (int q = 0; q < kPer; q += 4)
+          *reinterpret_cast<float4 *>(dst + q) =
+              make_float4(to_f32<Tin>(e[q]), to_f32<Tin>(e[q + 1]), to_f32<Tin>(e[q + 2]), to_f32<Tin>(e[q + 3]));
+        const size_t bh = bh0 + jh;
+        const int slot = (slot_n + j) % cap;
+        if (which == 0) {
           *reinterpret_cast<uint4 *>(kring + (bh * cap + slot) * DK + c) = raw;
-        } else {
-          const int cv = c - DK, hf = cv / HALF;
-          const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(vin + tok * DV + cv));
-          *reinterpret_cast<uint4 *>(vring + ((bh * 2 + hf) * cap + slot) * HALF + (cv - hf * HALF)) = raw;
+        } else if (which == 2) {
+          const int hf = c / HALF;
+          *reinterpret_cast<uint4 *>(vring + ((bh * 2 + hf) * cap + slot) * HALF + (c - hf * HALF)) = raw;
         }
       }
       named_sync(bar_id, kGroupThreads);
-      // ---- output scalars of every head (one warp per head), from the k rows of
-      //      the ring and the inputs: for output j (e = n + j) and window entry
-      //      i in [w0, e]: Mq_ji = e^{seg(i,e)} k_i.q_j, Mk_ji = e^{seg(i,e)} k_i.k_e
-      //      (i < e), 0 elsewhere; dec_j = e^{G}, G the g summed over [w0, e].
+      // ---- raw dots k_i.q_j and k_i.k_ej of every head and window entry i in
+      //      [w0, n + j] (the committed entries from the ring, the new ones from
+      //      shared memory)
       if (m > 0) {
-        constexpr int CE = MAXM == 1 ? 8 : 4;   // window entries per reduction
         constexpr int NV = CE * 2 * MAXM;
-        for (int jh = gw; jh < hc; jh += kGroupWarps) {
+        for (int t = gw; t < ntask; t += kGroupWarps) {
+          const int jh = t % hc, i0 = w0 + (t / hc) * CE;
           const size_t bh = bh0 + jh;
-          float *hs = hso + jh * HS::kOut;
-          float *hMk = hs + MAXM, *hMq = hMk + MAXM * 32;
-          float4 qv[MAXM], kv[MAXM];
+          float *hs = hso + jh * HSO;
+          float *hMk = hs + MAXM, *hMq = hMk + MAXM * kMaxW;
+          const float *hk = kqv + (size_t)jh * 3 * MAXM * DK, *hq = hk + MAXM * DK;
+          float part[NV];
 #pragma unroll
-          for (int j = 0; j < MAXM; ++j) {
-            const size_t tok = ((size_t)b * m + j) * a.H + h0 + jh;
-            qv[j] = j < m ? ld4<Tin>(qin + tok * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-            kv[j] = j < m ? ld4<Tin>(kin + tok * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-          for (int i0 = w0; i0 < ntot; i0 += CE) {
-            float part[NV];
-#pragma unroll
-            for (int c = 0; c < CE; ++c) {
-              const int i = i0 + c;
-              float4 ki = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (i < n)
-                ki = ld4<Tin>(kring + (bh * cap + (st + i) % cap) * DK + c0);
-              else if (i < ntot)
-                ki = ld4<Tin>(kin + (((size_t)b * m + (i - n)) * a.H + h0 + jh) * DK + c0);
-#pragma unroll
-              for (int j = 0; j < MAXM; ++j) {
-                part[(c * MAXM + j) * 2 + 0] = dot4(ki, qv[j]);
-                part[(c * MAXM + j) * 2 + 1] = dot4(ki, kv[j]);
-              }
+          for (int c = 0; c < CE; ++c) {
+            const int i = i0 + c;
+            float4 ki;
+            if (i < n) {
+              int slot = st + i;
+              if (slot >= cap) slot -= cap;
+              ki = ld4<Tin>(kring + (bh * cap + slot) * DK + c0);
+            } else if (i < ntot) {
+              ki = *reinterpret_cast<const float4 *>(hk + (i - n) * DK + c0);
+            } else {
+              ki = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            tr_sum<NV, 16>(part, lane);
-            const int base = tr_base<NV, 16>(lane);
-            constexpr int R = NV >= 32 ? NV / 32 : 1;
-            constexpr int DUP = NV >= 32 ? 1 : 32 / NV;
-            if ((lane & (DUP - 1)) == 0) {
 #pragma unroll
-              for (int q = 0; q < R; ++q) {   // raw dots, scaled below by their decays
-                const int idx = base + q, which = idx & 1, j = (idx >> 1) % MAXM, c = (idx >> 1) / MAXM;
-                const int l = i0 - w0 + c;
-                if (l < 32) (which == 0 ? hMq : hMk)[j * 32 + l] = part[q];
-              }
+            for (int j = 0; j < MAXM; ++j) {
+              const float4 qv = j < m ? *reinterpret_cast<const float4 *>(hq + j * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+              const float4 kv = j < m ? *reinterpret_cast<const float4 *>(hk + j * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+              part[(c * MAXM + j) * 2 + 0] = dot4(ki, qv);
+              part[(c * MAXM + j) * 2 + 1] = dot4(ki, kv);
             }
           }
-          __syncwarp();
-          const int l = lane, i = w0 + l;
+          tr_sum<NV, 16>(part, lane);
+          const int base = tr_base<NV, 16>(lane);
+          constexpr int R = NV >= 32 ? NV / 32 : 1;
+          constexpr int DUP = NV >= 32 ? 1 : 32 / NV;
+          if ((lane & (DUP - 1)) == 0) {
 #pragma unroll
-          for (int j = 0; j < MAXM; ++j) {
-            const int e = n + j, len = e - w0 + 1;
-            const float v = (j < m && l < len) ? sg[jh * WMAX + i] : 0.0f;
-            float after, total;
-            suffix_scan(v, lane, after, total);
-            const float ex = expf(after);
-            const bool in = j < m && l < len;
-            hMq[j * 32 + l] = in ? ex * hMq[j * 32 + l] : 0.0f;
-            hMk[j * 32 + l] = (in && l < len - 1) ? ex * hMk[j * 32 + l] : 0.0f;
-            if (lane == 0) hs[j] = j < m ? expf(total) : 0.0f;
+            for (int q = 0; q < R; ++q) {   // raw dots, scaled below by their decays
+              const int idx = base + q, which = idx & 1, j = (idx >> 1) % MAXM, c = (idx >> 1) / MAXM;
+              const int l = i0 - w0 + c;
+              if (l < kMaxW) (which == 0 ? hMq : hMk)[j * kMaxW + l] = part[q];
+            }
           }
+        }
+        named_sync(bar_id, kGroupThreads);
+        // ---- decays (one warp per head and token): for output j (e = n + j) and
+        //      window entry i in [w0, e]: Mq_ji = e^{seg(i,e)} k_i.q_j, Mk_ji =
+        //      e^{seg(i,e)} k_i.k_e (i < e), 0 elsewhere; dec_j = e^{G}, G the g
+        //      summed over [w0, e].
+        for (int t = gw; t < hc * MAXM; t += kGroupWarps) {
+          const int jh = t / MAXM, j = t - jh * MAXM;
+          float *hs = hso + jh * HSO;
+          float *hMk = hs + MAXM, *hMq = hMk + MAXM * kMaxW;
+          const int l = lane, e = n + j, len = e - w0 + 1;
+          const bool in = j < m && l < len;
+          const float v = in ? sg[jh * WMAX + w0 + l] : 0.0f;
+          float after, total;
+          suffix_scan(v, lane, after, total);
+          const float ex = expf(after);
+          hMq[j * kMaxW + l] = in ? ex * hMq[j * kMaxW + l] : 0.0f;
+          hMk[j * kMaxW + l] = (in && l < len - 1) ? ex * hMk[j * kMaxW + l] : 0.0f;
+          if (lane == 0) hs[j] = j < m ? expf(total) : 0.0f;
         }
       }
       named_sync(bar_id, kGroupThreads);
     }
 
-    // sequence number of this item's unit `unit` in the producer's issue order
-    const int pair = k >> 1;
-    const bool paired = 2 * pair + 1 < my_items;
-    const int seq0 = pair * 4 * hc + (paired ? (k & 1) : 0), step = paired ? 2 : 1;
-    int s = seq0 % stages, use = seq0 / stages;   // stage and use of the current unit
+    // stage and use of unit 2 jh + hf of this item, from its position in the
+    // producer's issue order
+    const IssueOrder<true> order(my_items, 2 * hc);
+    int s = 0, use = 0;
+    auto locate = [&](int jh, int hf) {
+      const int seq = order.seq(gi, k >> 1, 2 * jh + hf);
+      s = seq % stages;
+      use = seq / stages;
+    };
     auto wait_stage = [&]() -> bool {
       if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
       return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
@@ -480,13 +493,8 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     };
-    auto next_unit = [&]() {
-      s += step;
-      if (s >= stages) {
-        s -= stages;
-        ++use;
-      }
-    };
+    // fold windows: pre-fold = committed entries [0, n); window-full fold = [w0, n]
+    const int nf0 = n, nf1 = n - w0 + 1;
 
     // A failed wait (bounded, or another warp's abort) does not leave the loop:
     // the warp skips its work but passes every group barrier, whose OR
@@ -496,10 +504,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       const int h = h0 + jh;
       const size_t bh = bh0 + jh;
       const float *gw_ = sg + jh * WMAX, *bw_ = sbeta + jh * WMAX;
-      odec = hso + jh * HS::kOut;
-      Mk = odec + MAXM;
-      Mq = Mk + MAXM * 32;
-      for (int hf = 0; hf < 2; ++hf, next_unit()) {
+      const float *odec = hso + jh * HSO, *Mk = odec + MAXM, *Mq = Mk + MAXM * kMaxW;
+      const float *hk = kqv + (size_t)jh * 3 * MAXM * DK, *hq = hk + MAXM * DK, *hv = hq + MAXM * DK;
+      for (int hf = 0; hf < 2; ++hf) {
+        locate(jh, hf);
         if (rp.refuse) {
           if (!failed && wait_stage()) release_stage();
           else failed = true;
@@ -507,211 +515,342 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         }
         const size_t row_base = bh * DV + hf * HALF;   // first state row of this unit
         float *hc_rows = a.hc + row_base * DK;
-        uint8_t *rc = (RF != RSSM_READ_FP32) ? a.rc_codes + row_base * RB : nullptr;
-        float4 f[RPW];    // fp32 checkpoint rows for a fold (read-copy layers)
-        if constexpr (RF != RSSM_READ_FP32) {
+        uint8_t *rc = kResolve ? a.rc_codes + row_base * RB : nullptr;
+        float4 f[2][4];   // fp32 state rows (fp32 layers: the tile; re-solving layers: fold units)
+        if constexpr (kResolve) {
           if (pre || post) {
 #pragma unroll
-            for (int r = 0; r < RPW; ++r) f[r] = ld_stream(hc_rows + (size_t)(urow0 + r) * DK + c0);
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                f[r][c] = ld_stream(hc_rows + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8);
           }
         }
         // fold scalars are single-buffered: all warps must be done with the previous head's
         if (hf == 0 && (pre || post) && named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
         const bool have = !failed && wait_stage();
         if (!have) failed = true;
-        const GStage<Tin> stg{smem + s * stage_bytes, KOFF, QOFF, VOFF, WOFF, n, L};
+        bool released = false;
+        const uint8_t *sb = smem + s * Y.stage_bytes;
+        const float *wst = reinterpret_cast<const float *>(sb + Y.woff);   // cached w, committed entries
+        auto krow = [&](int i) -> const Tin * {
+          return reinterpret_cast<const Tin *>(sb + Y.koff) + (size_t)(i < n ? i : L + (i - n)) * DK;
+        };
+        auto vrow = [&](int i) -> const Tin * {
+          return reinterpret_cast<const Tin *>(sb + Y.voff) + (size_t)(i < n ? i : L + (i - n)) * HALF;
+        };
 
         if (hf == 0 && (pre || post)) {
-          // ---- fold scalars (fold heads only): Gram dots k_i'.k_i in 4 x 4 blocks.
+          // ---- fold scalars of this head
           if (have) {
-            const int nb = (nf + 3) / 4;
-            for (int blk = gw; blk < nb * nb; blk += kGroupWarps) {
-              const int bi = blk / nb, bj = blk - bi * nb;
-              if (bj > bi) continue;
-              float part[16];
-              float4 ka[4], kb[4];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int ia = 4 * bi + c, ib = 4 * bj + c;
-                ka[c] = ia < nf ? ld4<Tin>(stg.k(f0 + ia) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-                kb[c] = ib < nf ? ld4<Tin>(stg.k(f0 + ib) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-#pragma unroll
-              for (int ca = 0; ca < 4; ++ca)
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) part[ca * 4 + cb] = dot4(ka[ca], kb[cb]);
-              tr_sum<16, 16>(part, lane);
-              const int idx = tr_base<16, 16>(lane);
-              const int ia = 4 * bi + idx / 4, ib = 4 * bj + idx % 4;
-              if ((lane & 1) == 0 && ib < ia && ia < nf) {
-                // A[i][i'] = beta_i e^{seg(i', i)} k_i'.k_i (direct sums)
-                float sgm = 0.0f;
-                for (int r = ib + 1; r <= ia; ++r) sgm += gw_[f0 + r];
-                Mf[ia * kMaxW + ib] = bw_[f0 + ia] * expf(sgm) * part[0];
-              }
-            }
-            if (gw == 1 % kGroupWarps) {   // fold weights
-              const float v = lane < nf ? gw_[f0 + lane] : 0.0f;
+            if (gw == 1 && pre) {   // pre-fold window [0, n)
+              const float v = lane < nf0 ? gw_[lane] : 0.0f;
               float after, total;
               suffix_scan(v, lane, after, total);
               fw[lane] = expf(after);
               if (lane == 0) decF[0] = expf(total);
-              float pre_sum = 0.0f;   // e^{G_i}: g summed from the window start to entry i
-              for (int r = 0; r <= lane && r < nf; ++r) pre_sum += gw_[f0 + r];
-              decf[lane] = expf(pre_sum);
-              if (pre && post && lane == 0) {   // L = 1: then fold the new entry alone
-                one[0] = expf(gw_[n]);
-                one[1] = 1.0f;
-                one[2] = 1.0f;
+              if constexpr (kResolve) {
+                float ps = 0.0f;   // e^{G_i}: g summed from the window start through entry i
+                for (int r = 0; r <= lane && r < nf0; ++r) ps += gw_[r];
+                decf[lane] = expf(ps);
+              }
+            }
+            if (gw == 2 && post) {   // window-full fold [w0, n]
+              const float v = lane < nf1 ? gw_[w0 + lane] : 0.0f;
+              float after, total;
+              suffix_scan(v, lane, after, total);
+              fw[kMaxW + 1 + lane] = expf(after);
+              if (lane == 0) decF[1] = expf(total);
+              if constexpr (kResolve) {
+                float ps = 0.0f;
+                for (int r = 0; r <= lane && r < nf1; ++r) ps += gw_[w0 + r];
+                decf[kMaxW + 1 + lane] = expf(ps);
+              }
+            }
+            if constexpr (kResolve) {
+              // Gram dots of the re-solved window in 4 x 4 blocks:
+              // A[i][i'] = beta_i e^{seg(i', i)} k_i'.k_i (i' < i, direct sums).  A
+              // decode that folds twice (L = 1) re-solves two 1-entry windows (T = 1).
+              const int rf0 = pre ? 0 : w0, rnf = pre ? nf0 : nf1;
+              const int nb = (rnf + 3) / 4;
+              for (int blk = gw; blk < nb * nb; blk += kGroupWarps) {
+                const int bi = blk / nb, bj = blk - bi * nb;
+                if (bj > bi) continue;
+                float part[16];
+                float4 ka[4], kb[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  const int ia = 4 * bi + c, ib = 4 * bj + c;
+                  ka[c] = ia < rnf ? ld4<Tin>(krow(rf0 + ia) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  kb[c] = ib < rnf ? ld4<Tin>(krow(rf0 + ib) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int ca = 0; ca < 4; ++ca)
+#pragma unroll
+                  for (int cb = 0; cb < 4; ++cb) part[ca * 4 + cb] = dot4(ka[ca], kb[cb]);
+                tr_sum<16, 16>(part, lane);
+                const int idx = tr_base<16, 16>(lane);
+                const int ia = 4 * bi + idx / 4, ib = 4 * bj + idx % 4;
+                if ((lane & 1) == 0 && ib < ia && ia < rnf) {
+                  float sgm = 0.0f;
+                  for (int r = ib + 1; r <= ia; ++r) sgm += gw_[rf0 + r];
+                  Am[ia * L + ib] = bw_[rf0 + ia] * expf(sgm) * part[0];
+                }
               }
             }
           }
           if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
-          if (!failed && gw == 0) {
-            // T = (I + A)^{-1}: unit lower triangular, lane c computes column c
-            // by forward substitution (it reads only its own column of T).
-            const int c = lane;
-            for (int i = 0; i < nf; ++i) {
-              float v = i == c ? 1.0f : 0.0f;
-              if (i > c) {
-                float acc = 0.0f;
-                for (int ip = c; ip < i; ++ip) acc = fmaf(Mf[i * kMaxW + ip], Tm[ip * kMaxW + c], acc);
-                v = -acc;
+          if constexpr (kResolve) {
+            if (!failed && gw == 0) {
+              // T = (I + A)^{-1}: unit lower triangular, lane c computes column c
+              // by forward substitution (it reads only its own column of T).
+              const int rnf = pre ? nf0 : nf1, c = lane;
+              for (int i = 0; i < rnf; ++i) {
+                float v = i == c ? 1.0f : 0.0f;
+                if (i > c) {
+                  float acc = 0.0f;
+                  for (int ip = c; ip < i; ++ip) acc = fmaf(Am[i * L + ip], Tm[ip * L + c], acc);
+                  v = -acc;
+                }
+                if (c < rnf) Tm[i * L + c] = v;
               }
-              if (c < nf) Tm[i * kMaxW + c] = v;
             }
+            if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
           }
-          if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
         }
         if (failed) {
           if (have) release_stage();
           continue;
         }
 
-        // ---- the read view of this warp's 8 rows
-        float4 vw[RPW];
-        if (pre) {   // new tokens do not fit: fold the committed window first
-          if constexpr (RF == RSSM_READ_FP32) {
+        // ---- folds.  x <- decF x + sum_i fw_i w_i[row] k_i^T over the window
+        //      [i0, i0 + nf).  Layers that read the fp32 checkpoint take the w
+        //      cached in the ring (the new entry's from this warp's scratch);
+        //      re-solving layers first solve w from x by the UT transform:
+        //      u_i = x k_i, r_i = beta_i (v_i - e^{G_i} u_i), w = T r.
+        auto fold = [&](float4 (&x)[2][4], int i0, int nf, int which) {
+          const float *fwv = fw + which * (kMaxW + 1);
+          if constexpr (kResolve) {
+            const float *dfv = decf + which * (kMaxW + 1);
+            for (int ch = 0; ch < nf; ch += 4) {   // U[i][row] = x_row . k_i, 4 entries per reduction
+              float part[8];
 #pragma unroll
-            for (int r = 0; r < RPW; ++r)
-              f[r] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(urow0 + r) * DK + c0) * 4);
+              for (int c = 0; c < 4; ++c) {
+                const int i = ch + c;
+                float za = 0.0f, zb = 0.0f;
+                if (i < nf) {
+                  const Tin *kr = krow(i0 + i);
+#pragma unroll
+                  for (int cc = 0; cc < 4; ++cc) {
+                    const float4 k4 = ld4<Tin>(kr + 32 * cc + 4 * j8);
+                    za += dot4(x[0][cc], k4);
+                    zb += dot4(x[1][cc], k4);
+                  }
+                }
+                part[c] = za;
+                part[4 + c] = zb;
+              }
+              tr_sum<8, 4>(part, lane);
+              const int idx = tr_base<8, 4>(lane), r = idx >> 2, i = ch + (idx & 3);
+              if (i < nf) U[i * RPW + g8 + 4 * r] = part[0];
+            }
+            __syncwarp();
+            for (int p = lane; p < nf * RPW; p += 32) {   // r_i per (entry, row); U[i][r] layout
+              const int i = p / RPW, r8 = p - i * RPW;
+              U[p] = bw_[i0 + i] * fmaf(-dfv[i], U[p], to_f32<Tin>(vrow(i0 + i)[urow0 + r8]));
+            }
+            __syncwarp();
+            constexpr int kPer = kMaxW * RPW / 32;
+            float wv[kPer];
+            const float *Tw = (pre && post && which == 1) ? fwv : Tm;   // L = 1: T = 1 (= fw_0)
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+              const int p = lane + 32 * q, i = p / RPW, r8 = p - i * RPW;
+              float acc = 0.0f;
+              if (i < nf)
+                for (int ip = 0; ip <= i; ++ip) acc = fmaf(Tw[i * L + ip], U[ip * RPW + r8], acc);
+              wv[q] = acc;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < kPer; ++q)
+              if (lane + 32 * q < nf * RPW) U[lane + 32 * q] = wv[q];
+            __syncwarp();
           }
-          fold_rows<Tin>(f, stg, f0, nf, decf, Tm, fw, decF[0], bw_, urow0, U, lane, c0);
+          const float dF = decF[which];
 #pragma unroll
-          for (int r = 0; r < RPW; ++r) {
-            const int row = urow0 + r;
-            if (!post) st_stream(hc_rows + (size_t)row * DK + c0, f[r]);
-            if constexpr (RF == RSSM_READ_FP32)
-              vw[r] = f[r];
-            else
-              vw[r] = quantize4<RF, 32>(f[r], rc + (size_t)row * RB, a.rc_scales, row_base + row, DK, c0, lane);
-          }
-        } else {
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int r = 0; r < RPW; ++r) {
-            const int row = urow0 + r;
-            if constexpr (RF == RSSM_READ_FP32) {
-              vw[r] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)row * DK + c0) * 4);
-            } else if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
-              const uint32_t w = *reinterpret_cast<const uint32_t *>(stg.base + (size_t)row * RB + c0);
-              dec_e4m3x4(w, reinterpret_cast<const float *>(stg.base + TB)[row], vw[r]);
+            for (int c = 0; c < 4; ++c) scale4(x[r][c], dF);
+          for (int i = 0; i < nf; ++i) {
+            const int e = i0 + i;
+            float wa, wb;
+            if constexpr (kResolve) {
+              wa = U[i * RPW + g8];
+              wb = U[i * RPW + g8 + 4];
+            } else if (e < n) {
+              wa = wst[e * HALF + row_a];
+              wb = wst[e * HALF + row_b];
             } else {
-              const uint32_t w = *reinterpret_cast<const uint16_t *>(stg.base + (size_t)row * RB + c0 / 2);
-              const float sc = dec_e4m3(stg.base[TB + row * (DK / 16) + c0 / 16]);
-              dec_e2m1x4(w, sc, vw[r]);
+              wa = wnew[(e - n) * RPW + g8];
+              wb = wnew[(e - n) * RPW + g8 + 4];
+            }
+            const float cf = fwv[i];
+            wa *= cf;
+            wb *= cf;
+            const Tin *kr = krow(e);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float4 k4 = ld4<Tin>(kr + 32 * c + 4 * j8);
+              fma4(x[0][c], wa, k4);
+              fma4(x[1][c], wb, k4);
             }
           }
-        }
+          if constexpr (kResolve) __syncwarp();   // U is reused by the next fold
+        };
 
-        // ---- outputs.  Per row: z_j = dec_j (S k_ej) + sum_{committed i} Mk_ji w_i,
-        //      a_j = dec_j (S q_j) + sum_{committed i} Mq_ji w_i, reduced across
-        //      the row's lanes; then per row the new w and o in draft order.
-        if (m > 0) {
-          constexpr int NV = RPW * 2 * MAXM;
-          float part[NV];
+        // ---- the read view of this warp's rows, after a pre-fold if one is due
+        float4 v[2][4];   // read view (re-solving layers); fp32 layers read f
+        if constexpr (!kResolve) {
+          const float *tile = reinterpret_cast<const float *>(sb);
 #pragma unroll
-          for (int j = 0; j < MAXM; ++j) {
-            const float4 ke = j < m ? ld4<Tin>(stg.k(n + j) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 qj = j < m ? ld4<Tin>(stg.q(j) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float dj = odec[j < m ? j : 0];
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-            for (int r = 0; r < RPW; ++r) {
-              part[(r * MAXM + j) * 2 + 0] = dj * dot4(vw[r], ke);
-              part[(r * MAXM + j) * 2 + 1] = dj * dot4(vw[r], qj);
-            }
-          }
-          if (!pre && lane < n) {   // committed entry i = lane (w0 = 0)
-            float w8[RPW];
-            const float4 wa = reinterpret_cast<const float4 *>(stg.w(lane) + urow0)[0];
-            const float4 wb = reinterpret_cast<const float4 *>(stg.w(lane) + urow0)[1];
-            w8[0] = wa.x; w8[1] = wa.y; w8[2] = wa.z; w8[3] = wa.w;
-            w8[4] = wb.x; w8[5] = wb.y; w8[6] = wb.z; w8[7] = wb.w;
+            for (int c = 0; c < 4; ++c)
+              f[r][c] = *reinterpret_cast<const float4 *>(tile + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8);
+        }
+        if (pre) {   // the new tokens do not fit: fold the committed window first
+          fold(f, 0, nf0, 0);
 #pragma unroll
-            for (int j = 0; j < MAXM; ++j) {
-              const float mk = Mk[j * 32 + lane], mq = Mq[j * 32 + lane];
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-              for (int r = 0; r < RPW; ++r) {
-                part[(r * MAXM + j) * 2 + 0] = fmaf(mk, w8[r], part[(r * MAXM + j) * 2 + 0]);
-                part[(r * MAXM + j) * 2 + 1] = fmaf(mq, w8[r], part[(r * MAXM + j) * 2 + 1]);
+            for (int c = 0; c < 4; ++c)
+              if (!post) st_stream(hc_rows + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8, f[r][c]);
+          if constexpr (kResolve) quantize_rows<RF>(f, v, rc, a.rc_scales, row_base, row_a, row_b, j8, lane);
+        } else if constexpr (kResolve) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int row = r == 0 ? row_a : row_b;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(sb + (size_t)row * RB + 32 * c + 4 * j8);
+                dec_e4m3x4(w, reinterpret_cast<const float *>(sb + TB)[row], v[r][c]);
+              } else {
+                const uint32_t w = *reinterpret_cast<const uint16_t *>(sb + (size_t)row * RB + 16 * c + 2 * j8);
+                dec_e2m1x4(w, dec_e4m3(sb[TB + row * (DK / 16) + 2 * c + (j8 >> 2)]), v[r][c]);
               }
             }
           }
-          tr_sum<NV, 16>(part, lane);
-          const int base = tr_base<NV, 16>(lane);
-          constexpr int R = NV >= 32 ? NV / 32 : 1;
-          constexpr int DUP = NV >= 32 ? 1 : 32 / NV;
-          if constexpr (MAXM == 1) {
-            // one token: the lane holds z or a of its row; the other sits in lane ^ 2
-            const float other = __shfl_xor_sync(kFull, part[0], 2);
-            const int r = base >> 1, which = base & 1, row = urow0 + r, e = n;
-            const float z = which == 0 ? part[0] : other, av = which == 0 ? other : part[0];
-            const float wv = bw_[e] * (to_f32<Tin>(stg.v(e)[row]) - z);
-            if ((lane & 1) == 0) {
-              if (which == 0) wring[((bh * 2 + hf) * cap + (st + e) % cap) * HALF + row] = wv;
-              else a.out[((size_t)b * a.H + h) * DV + hf * HALF + row] = a.out_scale * fmaf(Mq[e - w0], wv, av);
-            }
-          } else {
-          if ((lane & (DUP - 1)) == 0) {
+        }
+
+        // ---- outputs.  Per row and token j: z = dec_j (S k_ej) + sum_i Mk_ji w_i,
+        //      a = dec_j (S q_j) + sum_i Mq_ji w_i over the committed entries i;
+        //      then per row the new w and o in draft order.
+        if (m > 0) {
+          float wz[MAXM], wa[MAXM];   // window sums: lane = (entry group lane >> 3, row lane & 7)
 #pragma unroll
-            for (int q = 0; q < R; ++q) red[base + q] = part[q];
+          for (int j = 0; j < MAXM; ++j) wz[j] = wa[j] = 0.0f;
+          if (!pre) {
+            for (int i = lane >> 3; i < n; i += 4) {
+              const float wv = wst[i * HALF + urow0 + (lane & 7)];
+#pragma unroll
+              for (int j = 0; j < MAXM; ++j) {
+                wz[j] = fmaf(Mk[j * kMaxW + i], wv, wz[j]);
+                wa[j] = fmaf(Mq[j * kMaxW + i], wv, wa[j]);
+              }
+            }
+          }
+          if (!post) {   // the last read of the stage: hand it back to the producer
+            release_stage();
+            released = true;
+          }
+          constexpr int NV = 4 * MAXM;   // (row r, token j, z|a) -> (r * MAXM + j) * 2 + which
+          float part[NV];
+#pragma unroll
+          for (int j = 0; j < MAXM; ++j) {
+            float za = 0.0f, zb = 0.0f, aa = 0.0f, ab = 0.0f;
+            if (j < m) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(hk + j * DK + 32 * c + 4 * j8);
+                const float4 q4 = *reinterpret_cast<const float4 *>(hq + j * DK + 32 * c + 4 * j8);
+                if constexpr (kResolve) {
+                  za += dot4(v[0][c], k4); zb += dot4(v[1][c], k4);
+                  aa += dot4(v[0][c], q4); ab += dot4(v[1][c], q4);
+                } else {
+                  za += dot4(f[0][c], k4); zb += dot4(f[1][c], k4);
+                  aa += dot4(f[0][c], q4); ab += dot4(f[1][c], q4);
+                }
+              }
+            }
+            part[j * 2 + 0] = za;
+            part[j * 2 + 1] = aa;
+            part[(MAXM + j) * 2 + 0] = zb;
+            part[(MAXM + j) * 2 + 1] = ab;
+          }
+#pragma unroll
+          for (int j = 0; j < MAXM; ++j) {   // sum the window terms over the 4 entry groups
+            wz[j] += __shfl_xor_sync(kFull, wz[j], 8);
+            wa[j] += __shfl_xor_sync(kFull, wa[j], 8);
+            wz[j] += __shfl_xor_sync(kFull, wz[j], 16);
+            wa[j] += __shfl_xor_sync(kFull, wa[j], 16);
+          }
+          tr_sum<NV, 4>(part, lane);   // over the 8 lanes of each row
+          {
+            const int base = tr_base<NV, 4>(lane);
+            constexpr int R = NV >= 8 ? NV / 8 : 1;
+            constexpr int DUP = NV >= 8 ? 1 : 8 / NV;
+            if ((lane & (DUP - 1)) == 0) {
+#pragma unroll
+              for (int q = 0; q < R; ++q) {
+                const int idx = base + q, r = idx / (2 * MAXM), jw = idx - r * 2 * MAXM;
+                red[(g8 + 4 * r) * 2 * MAXM + jw] = part[q];
+              }
+            }
+            if (lane < RPW) {
+#pragma unroll
+              for (int j = 0; j < MAXM; ++j) {
+                win[lane * 2 * MAXM + 2 * j + 0] = wz[j];
+                win[lane * 2 * MAXM + 2 * j + 1] = wa[j];
+              }
+            }
           }
           __syncwarp();
           if (lane < RPW) {
-            const int r = lane, row = urow0 + r;
+            const int r8 = lane, row = urow0 + r8;
             float wn[MAXM];
-            for (int j = 0; j < m; ++j) {
+#pragma unroll
+            for (int j = 0; j < MAXM; ++j) {
+              if (j >= m) break;
               const int e = n + j;
-              float acc = to_f32<Tin>(stg.v(e)[row]) - red[(r * MAXM + j) * 2 + 0];
-              for (int jp = 0; jp < j; ++jp) acc = fmaf(-Mk[j * 32 + (n + jp - w0)], wn[jp], acc);
+              const float dj = odec[j];
+              const float z = fmaf(dj, red[r8 * 2 * MAXM + 2 * j], win[r8 * 2 * MAXM + 2 * j]);
+              float acc = hv[j * DK + hf * HALF + row] - z;
+              for (int jp = 0; jp < j; ++jp) acc = fmaf(-Mk[j * kMaxW + (n + jp - w0)], wn[jp], acc);
               wn[j] = bw_[e] * acc;
-              float o = red[(r * MAXM + j) * 2 + 1];
-              for (int jp = 0; jp <= j; ++jp) o = fmaf(Mq[j * 32 + (n + jp - w0)], wn[jp], o);
+              float o = fmaf(dj, red[r8 * 2 * MAXM + 2 * j + 1], win[r8 * 2 * MAXM + 2 * j + 1]);
+              for (int jp = 0; jp <= j; ++jp) o = fmaf(Mq[j * kMaxW + (n + jp - w0)], wn[jp], o);
               a.out[(((size_t)b * m + j) * a.H + h) * DV + hf * HALF + row] = a.out_scale * o;
-              wring[((bh * 2 + hf) * cap + (st + e) % cap) * HALF + row] = wn[j];
+              int slot = slot_n + j;
+              if (slot >= cap) slot -= cap;
+              wring[((bh * 2 + hf) * cap + slot) * HALF + row] = wn[j];
+              wnew[j * RPW + r8] = wn[j];
             }
           }
           __syncwarp();
-          }
         }
 
-        if (post) {   // the decode filled the window: fold all of it (from fp32)
-          if constexpr (RF == RSSM_READ_FP32) {
+        if (post) {   // the decode filled the window: fold all of it
+          fold(f, w0, nf1, 1);
 #pragma unroll
-            for (int r = 0; r < RPW; ++r) f[r] = vw[r];
-          }
-          if (pre)   // L = 1: the window is the new entry alone
-            fold_rows<Tin>(f, stg, n, 1, one, one + 2, one + 1, one[0], bw_, urow0, U, lane, c0);
-          else
-            fold_rows<Tin>(f, stg, f0, nf, decf, Tm, fw, decF[0], bw_, urow0, U, lane, c0);
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int r = 0; r < RPW; ++r) {
-            const int row = urow0 + r;
-            st_stream(hc_rows + (size_t)row * DK + c0, f[r]);
-            if constexpr (RF != RSSM_READ_FP32)
-              quantize4<RF, 32>(f[r], rc + (size_t)row * RB, a.rc_scales, row_base + row, DK, c0, lane);
-          }
+            for (int c = 0; c < 4; ++c)
+              st_stream(hc_rows + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8, f[r][c]);
+          if constexpr (kResolve) quantize_rows<RF>(f, v, rc, a.rc_scales, row_base, row_a, row_b, j8, lane);
         }
-        release_stage();
+        if (!released) release_stage();
       }
     }
 
@@ -806,33 +945,38 @@ __global__ void __launch_bounds__(512) gdn_conv_kernel(const ConvArgs a) {
 
 template <typename Tin, int RF, int MAXM>
 cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
-  using HS = HeadScalars<MAXM>;
   auto kern = gdn_replay_kernel<Tin, RF, MAXM>;
-  const size_t esz = sizeof(Tin);
-  const size_t krow = DK * esz, vhrow = HALF * esz;
-  const size_t stage = ((size_t)tile_bytes<RF>() + scale_bytes<RF>() + (a.L + MAXM) * krow + MAXM * krow +
-                        (a.L + MAXM) * vhrow + (size_t)a.L * HALF * 4 + 127) & ~(size_t)127;
-  const size_t wmax = a.L + MAXM;
   int dev = 0, sms = 0, max_smem = 0;
   cudaError_t e;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   const size_t budget = (size_t)max_smem - 2048;
-  // heads per item: the largest divisor of H (at most 16) whose per-head scalars
-  // leave room for at least two stages
-  int hc = a.H < 16 ? a.H : 16;
-  size_t fixed = 0;
-  for (;; --hc) {
-    if (hc < 1) return cudaErrorInvalidConfiguration;
-    if (a.H % hc) continue;
-    const size_t group_floats = (2 * hc * wmax + (size_t)hc * HS::kOut + HS::kFold + kGroupWarps * HS::kWarp + 31) & ~(size_t)31;
-    fixed = kGroups * sizeof(float) * group_floats;
-    if (fixed + 2 * stage <= budget) break;
+  // Heads per item: among the divisors of H (at most 8) whose layout leaves room
+  // for two stages, prefer the deepest pipeline (up to 5 stages), then the
+  // fewest units on the busiest CTA (one CTA per SM), then the larger chunk.
+  int hc = 0, stages = 0;
+  long long best_units = 0;
+  for (int c = a.H < 8 ? a.H : 8; c >= 1; --c) {
+    if (a.H % c) continue;
+    const Layout y = make_layout<Tin, RF, MAXM>(a.L, c);
+    const size_t fixed = (size_t)kGroups * sizeof(float) * y.group_floats;
+    if (fixed + 2 * (size_t)y.stage_bytes > budget) continue;
+    int st = (int)((budget - fixed) / y.stage_bytes);
+    if (st > kMaxStages) st = kMaxStages;
+    const long long items = (long long)a.B * (a.H / c);
+    const long long units = (items + sms - 1) / sms * c;
+    const int depth = st < 5 ? st : 5;
+    const int best_depth = stages < 5 ? stages : 5;
+    if (hc == 0 || depth > best_depth || (depth == best_depth && units < best_units)) {
+      hc = c;
+      stages = st;
+      best_units = units;
+    }
   }
-  int stages = (int)((budget - fixed) / stage);
-  if (stages > kMaxStages) stages = kMaxStages;
-  const size_t smem = fixed + (size_t)stages * stage;
+  if (hc == 0) return cudaErrorInvalidConfiguration;
+  const Layout y = make_layout<Tin, RF, MAXM>(a.L, hc);
+  const size_t smem = (size_t)kGroups * sizeof(float) * y.group_floats + (size_t)stages * y.stage_bytes;
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   int per_sm = 0;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kReplayThreads, smem)) != cudaSuccess) return e;

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import seeded_inputs as si
-from gpu_common import DEV, GDN_KEYS, assert_close, dev_inputs, gdn_layer, rel_err, tok64
+from gpu_common import DEV, GDN_KEYS, assert_close, dev_inputs, gdn_layer, rel_err, to64, tok64
 from hybrid_ssm_decode_replayssm_b200 import rssm
 from oracle import bookkeeping as ob
 from oracle import codecs as oc
@@ -241,8 +241,11 @@ def test_quantized_reads_within_first_window(fmt):
 
 @pytest.mark.parametrize("fmt", FMTS)
 def test_read_copy_keeps_fp32_recurrence(fmt):
-    """The fp32 checkpoint trajectory is bit-identical with and without a read copy
-    (folds never use values read from it); the output error is reported."""
+    """The read copy serves only the reads: every fold of a read-copy layer solves
+    the window again from the fp32 checkpoint, so its checkpoint tracks the exact
+    state to fp32 rounding, like that of the fp32 layer (which folds with the w it
+    solved against the fp32 checkpoint while decoding).  The output error is
+    reported."""
     shape = si.GDNLayer(batch=3, nheads=4, dk=128, dv=128, window=8, dtype="bf16", state_std=0.05)
     lq, S0 = gdn_layer(shape, read_fmt=fmt)
     lf, _ = gdn_layer(shape)
@@ -252,10 +255,16 @@ def test_read_copy_keeps_fp32_recurrence(fmt):
     worst = 0.0
     for t in range(30):
         ins = dev_inputs(si.gdn_tokens(shape, t), GDN_KEYS)
+        before = lq.ckpt.clone()
         lq.decode_step(ins, oq)
         lf.decode_step(ins, of)
-        assert torch.equal(lq.ckpt, lf.ckpt), f"fp32 checkpoints diverged at step {t}"
         S, o = _oracle_step(S, si.gdn_tokens(shape, t))
+        if (t + 1) % 8 == 0:   # the window filled: both layers folded
+            assert_close(lq.ckpt.cpu(), S, TOL["f32"], f"read-copy checkpoint after step {t}")
+            assert_close(lf.ckpt.cpu(), S, TOL["f32"], f"fp32 checkpoint after step {t}")
+            assert_close(lq.ckpt.cpu(), to64(lf.ckpt), 1e-5, f"checkpoints apart after step {t}")
+        else:
+            assert torch.equal(lq.ckpt, before), f"checkpoint written at step {t}"
         worst = max(worst, rel_err(oq.cpu(), o))
     assert worst < (0.1 if fmt == rssm.RSSM_READ_FP8_E4M3_ROW else 0.5)
     print(f"read copy {fmt}: max scaled output error {worst:.3e}")
