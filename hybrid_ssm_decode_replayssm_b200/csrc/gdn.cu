@@ -25,11 +25,12 @@
 // Work unit: half a head (64 of the 128 value rows, 32 KiB of fp32 state).  A
 // persistent CTA has one producer warp, which streams units into a ring of
 // shared-memory stages with 1-D TMA bulk copies (the read tile and the cached
-// w rows; fold units also the window's k and v rows), and two consumer groups
-// of 8 warps taking alternate items (item = one sequence and a chunk of
+// w rows; fold units of re-solving layers also the v rows), and two consumer
+// groups of 8 warps taking alternate items (item = one sequence and a chunk of
 // heads), whose units the producer interleaves (IssueOrder).  An item's
-// prologue converts the new q, k, v rows to fp32 in shared memory, appends k
-// and v to the ring and computes every head's window scalars.  Per unit each warp owns 8 state rows; a row is spread over 8
+// prologue copies the committed window k rows of its heads into shared memory
+// (cp.async), loads the gates, converts the new q, k, v rows to fp32, appends
+// to the ring and computes every head's window scalars.  Per unit each warp owns 8 state rows; a row is spread over 8
 // lanes (4 chunks of 4 columns each), so its dot products reduce in three
 // shuffle steps.
 #include "rssm_device.cuh"
@@ -76,28 +77,29 @@ __device__ __forceinline__ void scale4(float4 &t, float c) { t.x *= c; t.y *= c;
 
 // Shared-memory layout of a replay launch (the host sizes the launch with the
 // same function).  Stage, in bytes: [read tile | scales | cached w rows (L) |
-// k rows (L + MAXM, fold units) | v half rows (L + MAXM, fold units of
-// re-solving layers)]; committed entries at rows [0, n), new tokens at L + j.
-// Group region, in floats: gates and betas of the item's heads, fp32 k/q/v of
-// the new tokens, per-head output scalars, fold scalars, per-warp scratch.
+// v half rows (L + MAXM, fold units of re-solving layers; committed entries
+// at rows [0, n), new tokens at L + j)].  Group region, in floats: gates and
+// betas of the item's heads, fp32 k/q/v of the new tokens, the committed
+// window k rows of the item's heads (input dtype), per-head output scalars,
+// fold scalars, per-warp scratch.
 struct Layout {
-  int woff, koff, voff, stage_bytes;
-  int sg, sbeta, kqv, hso, fold, warp, warp_floats, group_floats;
+  int woff, voff, stage_bytes;
+  int sg, sbeta, kqv, kbuf, hso, fold, warp, warp_floats, group_floats;
 };
 template <typename Tin, int RF, int MAXM>
 __host__ __device__ inline Layout make_layout(int L, int hc) {
   constexpr bool kResolve = RF != RSSM_READ_FP32;
   Layout y;
-  const int krow = DK * (int)sizeof(Tin), vhrow = HALF * (int)sizeof(Tin);
+  const int vhrow = HALF * (int)sizeof(Tin);
   y.woff = tile_bytes<RF>() + scale_bytes<RF>();
-  y.koff = y.woff + L * HALF * 4;
-  y.voff = y.koff + (L + MAXM) * krow;
+  y.voff = y.woff + L * HALF * 4;
   y.stage_bytes = (y.voff + (kResolve ? (L + MAXM) * vhrow : 0) + 127) & ~127;
   const int wmax = L + MAXM;
   y.sg = 0;
   y.sbeta = hc * wmax;
   y.kqv = (2 * hc * wmax + 3) & ~3;
-  y.hso = y.kqv + hc * 3 * MAXM * DK;
+  y.kbuf = y.kqv + hc * 3 * MAXM * DK;   // [hc][L][DK] input dtype, 16-byte aligned
+  y.hso = y.kbuf + hc * L * DK * (int)sizeof(Tin) / 4;
   y.fold = y.hso + hc * (MAXM + 2 * MAXM * kMaxW);
   // fw[2][kMaxW + 1] | decF[2] | decf[2][kMaxW + 1] | A[L][L] | T[L][L] (A, T: re-solving layers)
   const int fold_floats = 4 * (kMaxW + 1) + 2 + (kResolve ? 2 * L * L : 0);
@@ -180,7 +182,6 @@ template <typename Tin, int RF, int MAXM>
 __global__ void __launch_bounds__(kReplayThreads, 1)
     gdn_replay_kernel(const StepArgs a, const int hc, const int stages) {
   constexpr bool kResolve = RF != RSSM_READ_FP32;
-  constexpr int KROW = DK * (int)sizeof(Tin);
   constexpr int VHROW = HALF * (int)sizeof(Tin);
   constexpr int TB = tile_bytes<RF>();
   constexpr int SB = scale_bytes<RF>();
@@ -269,11 +270,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         // cached w rows: the reads of the committed entries, and the folds of
         // layers that fold with them
         const int nw = (kResolve && rp.pre) ? 0 : rp.n;
-        const int nk = fold ? rp.n : 0;                       // k rows of fold units
         const int nv = (kResolve && fold) ? rp.n : 0;         // v rows of re-solving folds
-        const int mk = fold ? m : 0, mv = (kResolve && fold) ? m : 0;
+        const int mv = (kResolve && fold) ? m : 0;
         uint8_t *dst = smem + s * Y.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + nw * HALF * 4 + (nk + mk) * KROW + (nv + mv) * VHROW));
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + nw * HALF * 4 + (nv + mv) * VHROW));
         if constexpr (RF == RSSM_READ_FP32) {
           bulk_g2s(dst, a.hc + (bh * DV + hf * HALF) * DK, TB, &full[s]);
         } else {
@@ -287,20 +287,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           bulk_g2s(dst + Y.woff, src + (size_t)rp.st * HALF, w1 * HALF * 4, &full[s]);
           if (nw > w1) bulk_g2s(dst + Y.woff + w1 * HALF * 4, src, (nw - w1) * HALF * 4, &full[s]);
         }
-        if (nk > 0) {
-          const Tin *src = kring + bh * cap * DK;
-          bulk_g2s(dst + Y.koff, src + (size_t)rp.st * DK, c1 * KROW, &full[s]);
-          if (nk > c1) bulk_g2s(dst + Y.koff + c1 * KROW, src, (nk - c1) * KROW, &full[s]);
-        }
         if (nv > 0) {
           const Tin *src = vring + (bh * 2 + hf) * cap * HALF;
           bulk_g2s(dst + Y.voff, src + (size_t)rp.st * HALF, c1 * VHROW, &full[s]);
           if (nv > c1) bulk_g2s(dst + Y.voff + c1 * VHROW, src, (nv - c1) * VHROW, &full[s]);
         }
-        for (int j = 0; j < mk; ++j) {
+        for (int j = 0; j < mv; ++j) {
           const size_t tok = ((size_t)b * m + j) * a.H + h;
-          bulk_g2s(dst + Y.koff + (L + j) * KROW, kin + tok * DK, KROW, &full[s]);
-          if (j < mv) bulk_g2s(dst + Y.voff + (L + j) * VHROW, vin + tok * DV + hf * HALF, VHROW, &full[s]);
+          bulk_g2s(dst + Y.voff + (L + j) * VHROW, vin + tok * DV + hf * HALF, VHROW, &full[s]);
         }
       }
       *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
@@ -323,6 +317,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   float *sg = G + Y.sg;          // [hc][WMAX]  ln alpha of the window entries
   float *sbeta = G + Y.sbeta;    // [hc][WMAX]
   float *kqv = G + Y.kqv;        // [hc][k | q | v][MAXM][128]  new tokens, fp32
+  Tin *kbuf = reinterpret_cast<Tin *>(G + Y.kbuf);   // [hc][L][128]  committed window k rows
   float *hso = G + Y.hso;        // [hc][HSO]
   float *fw = G + Y.fold;        // [2][kMaxW + 1]  fold weights e^{seg(i, last)}: pre-fold, window-full fold
   float *decF = fw + 2 * (kMaxW + 1);   // [2]  decay over each fold window
@@ -352,13 +347,16 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     const int slot_n = (st + n) % cap;   // ring slot of the first new entry
 
     if (!rp.refuse) {
-      // Window scalars are computed in tasks (head jh, batch of CE window
-      // entries) spread over the group's warps.  (Loading a task's ring k rows
-      // before the first barrier was measured slower: the registers it holds
-      // across the barrier spill.)
-      constexpr int CE = MAXM == 1 ? 8 : 4;   // window entries per reduction
-      const int nbatch = m > 0 ? (ntot - w0 + CE - 1) / CE : 0;
-      const int ntask = hc * nbatch;
+      // ---- committed window k rows of the item's heads into shared memory
+      //      (asynchronous copies, in flight while the loads below are made)
+      constexpr int kChunks = DK * (int)sizeof(Tin) / 16;   // 16-byte chunks per row
+      for (int idx = gt; idx < hc * n * kChunks; idx += kGroupThreads) {
+        const int c = idx % kChunks, r = idx / kChunks;
+        const int i = r % n, jh = r / n;
+        const int slot = (st + i) % cap;
+        cp_async16(reinterpret_cast<uint8_t *>(kbuf + ((size_t)jh * L + i) * DK) + 16 * c,
+                   reinterpret_cast<const uint8_t *>(kring + ((bh0 + jh) * cap + slot) * DK) + 16 * c);
+      }
       // ---- gates and betas of the item's heads; ring appends of the new gates
       for (int idx = gt; idx < hc * ntot; idx += kGroupThreads) {
         const int jh = idx / ntot, i = idx - jh * ntot;
@@ -406,32 +404,28 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           *reinterpret_cast<uint4 *>(vring + ((bh * 2 + hf) * cap + slot) * HALF + (c - hf * HALF)) = raw;
         }
       }
+      cp_async_wait_all();
       named_sync(bar_id, kGroupThreads);
       // ---- raw dots k_i.q_j and k_i.k_ej of every head and window entry i in
-      //      [w0, n + j] (the committed entries from the ring, the new ones from
-      //      shared memory)
+      //      [w0, n + j], in tasks (head, batch of CE entries) over the warps
       if (m > 0) {
+        constexpr int CE = MAXM == 1 ? 8 : 4;   // window entries per reduction
         constexpr int NV = CE * 2 * MAXM;
-        for (int t = gw; t < ntask; t += kGroupWarps) {
+        const int nbatch = (ntot - w0 + CE - 1) / CE;
+        for (int t = gw; t < hc * nbatch; t += kGroupWarps) {
           const int jh = t % hc, i0 = w0 + (t / hc) * CE;
-          const size_t bh = bh0 + jh;
-          float *hs = hso + jh * HSO;
-          float *hMk = hs + MAXM, *hMq = hMk + MAXM * kMaxW;
+          float *hMk = hso + jh * HSO + MAXM, *hMq = hMk + MAXM * kMaxW;
           const float *hk = kqv + (size_t)jh * 3 * MAXM * DK, *hq = hk + MAXM * DK;
+          const Tin *kb = kbuf + (size_t)jh * L * DK;
           float part[NV];
 #pragma unroll
           for (int c = 0; c < CE; ++c) {
             const int i = i0 + c;
-            float4 ki;
-            if (i < n) {
-              int slot = st + i;
-              if (slot >= cap) slot -= cap;
-              ki = ld4<Tin>(kring + (bh * cap + slot) * DK + c0);
-            } else if (i < ntot) {
+            float4 ki = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < n)
+              ki = ld4<Tin>(kb + (size_t)i * DK + c0);
+            else if (i < ntot)
               ki = *reinterpret_cast<const float4 *>(hk + (i - n) * DK + c0);
-            } else {
-              ki = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
 #pragma unroll
             for (int j = 0; j < MAXM; ++j) {
               const float4 qv = j < m ? *reinterpret_cast<const float4 *>(hq + j * DK + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -472,8 +466,8 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           hMk[j * kMaxW + l] = (in && l < len - 1) ? ex * hMk[j * kMaxW + l] : 0.0f;
           if (lane == 0) hs[j] = j < m ? expf(total) : 0.0f;
         }
+        named_sync(bar_id, kGroupThreads);
       }
-      named_sync(bar_id, kGroupThreads);
     }
 
     // stage and use of unit 2 jh + hf of this item, from its position in the
@@ -533,15 +527,18 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         bool released = false;
         const uint8_t *sb = smem + s * Y.stage_bytes;
         const float *wst = reinterpret_cast<const float *>(sb + Y.woff);   // cached w, committed entries
-        auto krow = [&](int i) -> const Tin * {
-          return reinterpret_cast<const Tin *>(sb + Y.koff) + (size_t)(i < n ? i : L + (i - n)) * DK;
+        const Tin *kb = kbuf + (size_t)jh * L * DK;
+        // k_i[col .. col + 3]: committed entries from the item's k rows, new ones (fp32)
+        auto kval4 = [&](int i, int col) -> float4 {
+          return i < n ? ld4<Tin>(kb + (size_t)i * DK + col) : *reinterpret_cast<const float4 *>(hk + (i - n) * DK + col);
         };
         auto vrow = [&](int i) -> const Tin * {
           return reinterpret_cast<const Tin *>(sb + Y.voff) + (size_t)(i < n ? i : L + (i - n)) * HALF;
         };
 
         if (hf == 0 && (pre || post)) {
-          // ---- fold scalars of this head
+          // ---- fold scalars of this head: weights and decays of both fold
+          //      windows, and the Gram dots of a re-solved window
           if (have) {
             if (gw == 1 && pre) {   // pre-fold window [0, n)
               const float v = lane < nf0 ? gw_[lane] : 0.0f;
@@ -577,17 +574,17 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
                 const int bi = blk / nb, bj = blk - bi * nb;
                 if (bj > bi) continue;
                 float part[16];
-                float4 ka[4], kb[4];
+                float4 ka[4], kb_[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                   const int ia = 4 * bi + c, ib = 4 * bj + c;
-                  ka[c] = ia < rnf ? ld4<Tin>(krow(rf0 + ia) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-                  kb[c] = ib < rnf ? ld4<Tin>(krow(rf0 + ib) + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  ka[c] = ia < rnf ? kval4(rf0 + ia, c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  kb_[c] = ib < rnf ? kval4(rf0 + ib, c0) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
                 for (int ca = 0; ca < 4; ++ca)
 #pragma unroll
-                  for (int cb = 0; cb < 4; ++cb) part[ca * 4 + cb] = dot4(ka[ca], kb[cb]);
+                  for (int cb = 0; cb < 4; ++cb) part[ca * 4 + cb] = dot4(ka[ca], kb_[cb]);
                 tr_sum<16, 16>(part, lane);
                 const int idx = tr_base<16, 16>(lane);
                 const int ia = 4 * bi + idx / 4, ib = 4 * bj + idx % 4;
@@ -639,10 +636,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
                 const int i = ch + c;
                 float za = 0.0f, zb = 0.0f;
                 if (i < nf) {
-                  const Tin *kr = krow(i0 + i);
 #pragma unroll
                   for (int cc = 0; cc < 4; ++cc) {
-                    const float4 k4 = ld4<Tin>(kr + 32 * cc + 4 * j8);
+                    const float4 k4 = kval4(i0 + i, 32 * cc + 4 * j8);
                     za += dot4(x[0][cc], k4);
                     zb += dot4(x[1][cc], k4);
                   }
@@ -698,10 +694,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             const float cf = fwv[i];
             wa *= cf;
             wb *= cf;
-            const Tin *kr = krow(e);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const float4 k4 = ld4<Tin>(kr + 32 * c + 4 * j8);
+              const float4 k4 = kval4(e, 32 * c + 4 * j8);
               fma4(x[0][c], wa, k4);
               fma4(x[1][c], wb, k4);
             }
@@ -952,11 +947,13 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   const size_t budget = (size_t)max_smem - 2048;
-  // Heads per item: among the divisors of H (at most 8) whose layout leaves room
-  // for two stages, prefer the deepest pipeline (up to 5 stages), then the
-  // fewest units on the busiest CTA (one CTA per SM), then the larger chunk.
+  // Heads per item: the divisor of H (at most 8) with the lowest cost on the
+  // busiest CTA (one CTA per SM): its items times (2 units per head + about 4
+  // units' worth of item prologue, which both consumer groups run at the same
+  // time), raised when the layout leaves fewer than 4 stages.  Measured at
+  // batch 256: 8 heads per item (4 stages) beat 2 heads (5 stages) by 14%.
   int hc = 0, stages = 0;
-  long long best_units = 0;
+  double best_cost = 0.0;
   for (int c = a.H < 8 ? a.H : 8; c >= 1; --c) {
     if (a.H % c) continue;
     const Layout y = make_layout<Tin, RF, MAXM>(a.L, c);
@@ -965,13 +962,12 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
     int st = (int)((budget - fixed) / y.stage_bytes);
     if (st > kMaxStages) st = kMaxStages;
     const long long items = (long long)a.B * (a.H / c);
-    const long long units = (items + sms - 1) / sms * c;
-    const int depth = st < 5 ? st : 5;
-    const int best_depth = stages < 5 ? stages : 5;
-    if (hc == 0 || depth > best_depth || (depth == best_depth && units < best_units)) {
+    double cost = (double)((items + sms - 1) / sms) * (2 * c + 4);
+    if (st < 4) cost *= 4.0 / st;
+    if (hc == 0 || cost < best_cost) {
       hc = c;
       stages = st;
-      best_units = units;
+      best_cost = cost;
     }
   }
   if (hc == 0) return cudaErrorInvalidConfiguration;

@@ -313,6 +313,16 @@ __device__ __forceinline__ bool wait_flag_at_least(const int *flag, int value, v
   return true;
 }
 
+// Asynchronous 16-byte global -> shared copies (cp.async, L1 bypassed): issued
+// without holding registers; a thread's copies are complete after
+// cp_async_wait_all(), and visible to the other threads after a barrier.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Named barrier `id` (1..15) over `n` threads (a group of consumer warps of a
 // warp-specialised CTA), optionally OR-reducing a predicate.
 __device__ __forceinline__ void named_sync(int id, int n) {
