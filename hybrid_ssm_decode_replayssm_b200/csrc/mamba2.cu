@@ -79,7 +79,7 @@ struct Stage {
   }
 };
 
-// t <- dec * t + sum_{i0 <= i < i1} fw[i - i0] x_i[row] B_i[cols]   (rank-(i1-i0) fold)
+// t <- dec * t + sum_{i0 <= i < i1} x_i[row] (fw[i - i0] B_i[cols])   (rank-(i1-i0) fold)
 template <int P, int N, int W, typename Tin>
 __device__ __forceinline__ void fold_tile(float4 (&t)[Tile<P, N, W>::NLD], const float *s_fw, float dec,
                                           int i0, int i1, const Stage &stg, const float *s_B,
@@ -90,15 +90,17 @@ __device__ __forceinline__ void fold_tile(float4 (&t)[Tile<P, N, W>::NLD], const
     t[l].x *= dec; t[l].y *= dec; t[l].z *= dec; t[l].w *= dec;
   }
   for (int i = i0; i < i1; ++i) {
-    const float4 bv = *reinterpret_cast<const float4 *>(s_B + i * N + c0);
     const float fw = s_fw[i - i0];
+    float4 bv = *reinterpret_cast<const float4 *>(s_B + i * N + c0);
+    bv.x *= fw; bv.y *= fw; bv.z *= fw; bv.w *= fw;
+    float xr[T::NLD];
+    stg.xs<Tin, T::NLD>(i, row0, T::RPI, xr);   // this lane's rows: one vector load when contiguous
 #pragma unroll
     for (int l = 0; l < T::NLD; ++l) {
-      const float xr = fw * stg.x<Tin>(i, row0 + l * T::RPI);
-      t[l].x = fmaf(xr, bv.x, t[l].x);
-      t[l].y = fmaf(xr, bv.y, t[l].y);
-      t[l].z = fmaf(xr, bv.z, t[l].z);
-      t[l].w = fmaf(xr, bv.w, t[l].w);
+      t[l].x = fmaf(xr[l], bv.x, t[l].x);
+      t[l].y = fmaf(xr[l], bv.y, t[l].y);
+      t[l].z = fmaf(xr[l], bv.z, t[l].z);
+      t[l].w = fmaf(xr[l], bv.w, t[l].w);
     }
   }
 }
@@ -191,11 +193,13 @@ constexpr int kGroupThreads = kGroupWarps * 32;
 constexpr int kConsumers = kGroups * kGroupThreads;
 constexpr int kReplayThreads = kConsumers + 32; // + one producer warp
 constexpr int kMaxStages = 16;
+constexpr int kPairSlots = 32;                  // > 1 + kMaxStages / 2 pairs in flight
 
 // The replay kernel: persistent and warp-specialised.  CTA c works through the
 // items c, c + grid, ... where an item is one (sequence b, group g, chunk of
-// `hc` heads); its heads are numbered in one sequence across the CTA's items
-// (seq = k * hc + jh), stage = seq % stages, use u = seq / stages.
+// `hc` heads); consumer group k % 2 takes item k.  The heads of the CTA's
+// items are numbered in the producer's issue order (seq: pairs of items, see
+// the producer), stage = seq % stages, use u = seq / stages.
 //  * Producer warp (one lane): for each head in sequence, waits until the
 //    consumers have released its stage (empty barrier, phase u - 1), then
 //    requests with 1-D TMA bulk copies the head's read tile (fp32, or FP8/NVFP4
@@ -225,6 +229,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   // further ahead, so it first waits for stage_use[s] == u.
   __shared__ int stage_use[kMaxStages];
   __shared__ int abort_flag;
+  // pair_inter[p % kPairSlots]: the heads of the CTA's items 2p and 2p + 1
+  // alternate in the issue order (both items fold).  The producer decides it
+  // before issuing the pair's first head, when no item of the pair has been
+  // processed (so the pair's ring pointers cannot have moved), and publishes
+  // it before that head's stage_use; a consumer reads it after seeing that
+  // stage_use.  The producer cannot run kPairSlots pairs ahead of a reader:
+  // it stays within `stages` heads of the oldest unreleased one.
+  __shared__ int pair_inter[kPairSlots];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L, cap = a.cap, m = a.m, WMAX = L + MAXM;
@@ -244,6 +256,13 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   Tin *xring = reinterpret_cast<Tin *>(a.buf0);
   volatile int *abort = &abort_flag;
 
+  auto item_of = [&](int k, int &b, int &g, int &chunk) {
+    const int item = (int)blockIdx.x + k * (int)gridDim.x;
+    b = item / (a.G * nchunk);
+    const int rem = item - b * a.G * nchunk;
+    g = rem / nchunk;
+    chunk = rem - g * nchunk;
+  };
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
@@ -255,31 +274,46 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   }
   __syncthreads();
 
-  auto item_of = [&](int k, int &b, int &g, int &chunk) {
-    const int item = (int)blockIdx.x + k * (int)gridDim.x;
-    b = item / (a.G * nchunk);
-    const int rem = item - b * a.G * nchunk;
-    g = rem / nchunk;
-    chunk = rem - g * nchunk;
-  };
-
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    int cur_k = -1, b = 0, g = 0, chunk = 0, jh = 0, s = 0, u = 0;
-    RowPlan rp{};
+    // Issue order, per pair of items (2p, 2p + 1): the heads of item 2p, then of
+    // item 2p + 1 (one group's item prologue overlaps the other group's heads);
+    // when both items fold, their heads alternate so that both groups compute.
+    int p = 0, w = 0;   // pair and position in the pair of unit seq
+    int cur_p = -1, b = 0, g = 0, chunk = 0, jh = 0, s = 0, u = 0, b_o = 0, g_o = 0, chunk_o = 0;
+    bool inter = false;
+    RowPlan rp{}, rp_e{}, rp_o{};   // current item; the pair's even and odd items
+    int b_e = 0, g_e = 0, chunk_e = 0;
     int issued = 0;
     for (int seq = 0; seq < total_seq; ++seq) {
       if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
         atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
         break;
       }
-      if (cur_k < 0 || jh == hc) {
-        ++cur_k;
-        jh = 0;
-        item_of(cur_k, b, g, chunk);
-        rp = plan_row(a, b);
+      if (w == 2 * hc) {   // next pair
+        w = 0;
+        ++p;
       }
+      if (p != cur_p) {
+        cur_p = p;
+        item_of(2 * p, b_e, g_e, chunk_e);
+        rp_e = plan_row(a, b_e);
+        const bool has_odd = 2 * p + 1 < my_items;
+        if (has_odd) {
+          item_of(2 * p + 1, b_o, g_o, chunk_o);
+          rp_o = plan_row(a, b_o);
+        }
+        inter = has_odd && (rp_e.pre || rp_e.post) && (rp_o.pre || rp_o.post);
+        *reinterpret_cast<volatile int *>(&pair_inter[p % kPairSlots]) = inter ? 1 : 0;
+        __threadfence_block();   // visible before this head's stage_use
+      }
+      const bool odd = inter ? (w & 1) != 0 : w >= hc;
+      jh = inter ? (w >> 1) : (odd ? w - hc : w);
+      b = odd ? b_o : b_e;
+      g = odd ? g_o : g_e;
+      chunk = odd ? chunk_o : chunk_e;
+      rp = odd ? rp_o : rp_e;
       issued = seq + 1;
       if (rp.refuse) {
         mbar_arrive(&full[s]);
@@ -304,7 +338,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           bulk_g2s(dst + XOFF + (L + j) * XROW, xin + (((size_t)b * m + j) * a.H + h) * P, XROW, &full[s]);
       }
       *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
-      ++jh;
+      ++w;
       if (++s == stages) {
         s = 0;
         ++u;
@@ -425,16 +459,33 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       named_sync(bar_id, kGroupThreads);
     }
 
-    // ---- heads: every warp of the group works on its rows
-    int s = (k * hc) % stages;
-    int use = (k * hc) / stages;
+    // ---- heads: every warp of the group works on its rows.  Head jh is number
+    //      2 p hc + (2 jh + (k & 1) | (k & 1) hc + jh) in the producer's issue
+    //      order (p = k / 2; interleaved when both items of the pair fold).
+    const int seq_base = (k >> 1) * 2 * hc;
+    int s = seq_base % stages, use = seq_base / stages;
+    bool inter = false;
+    if (wait_flag_at_least(&stage_use[s], use, abort)) {   // the pair's first head is issued
+      __threadfence_block();
+      inter = *reinterpret_cast<volatile int *>(&pair_inter[(k >> 1) % kPairSlots]) != 0;
+    }
     // wait until the producer has requested use `use` of stage s, then for the data
     auto wait_stage = [&]() -> bool {
       if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
       return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
     };
-    for (int jh = 0; jh < hc; ++jh) {
+    {
+      const int seq = seq_base + (inter ? (k & 1) : (k & 1) * hc);   // the item's first head
+      s = seq % stages;
+      use = seq / stages;
+    }
+    const int step = inter ? 2 : 1;
+    for (int jh = 0; jh < hc; ++jh, s += step) {
       const int h = h0 + jh;
+      if (s >= stages) {
+        s -= stages;
+        ++use;
+      }
       if (rp.refuse) {
         if (!wait_stage()) break;
       } else {
@@ -506,10 +557,6 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);   // this warp is done with stage s
-      if (++s == stages) {
-        s = 0;
-        ++use;
-      }
     }
 
     // ---- item end: the group's warps are done; the last CTA of sequence b
