@@ -187,6 +187,40 @@ __device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
   return r;
 }
 
+// Decode heads of read-copy layers (bf16 inputs, headdim 64, dstate 128) take
+// the tensor-core path: y = h C as mma.sync m16n8k16 (f16 x f16 -> fp32), one
+// warp per 16-row tile, four warps per head.  The dequantised codes are exact
+// in f16 (an E2M1 value times an E4M3 scale has at most 6 significant bits and
+// lies in [2^-10, 2688]; an E4M3 code is exact and its fp32 row scale is
+// applied to the result); C is scaled by a power of two so that max |C| lies
+// in [2^14, 2^15) before rounding to f16, which keeps every bf16 bit of the
+// values within 2^15 of the largest.  The products are exact in fp32.
+template <int P, int N, typename Tin, int RF, int MAXM>
+constexpr bool mma_read() {
+  return RF != RSSM_READ_FP32 && sizeof(Tin) == 2 && MAXM == 1 && P == 64 && N == 128;
+}
+template <int P, int N, typename Tin, int RF, int MAXM>
+constexpr int mma_floats() { return mma_read<P, N, Tin, RF, MAXM>() ? N / 2 + 4 : 0; }   // C as f16, 1/scale
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t h2bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
+// two E2M1 codes (one byte, element 0 in the low nibble) -> f16x2, times a f16x2 scale
+__device__ __forceinline__ uint32_t e2m1x2_scaled(uint32_t byte, __half2 sc) {
+  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xFFu), __NV_E2M1);
+  return h2bits(__hmul2(__half2(r), sc));
+}
+// two E4M3 codes (16 bits, element 0 in the low byte) -> f16x2
+__device__ __forceinline__ uint32_t e4m3x2_h2(uint32_t bits) {
+  const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(bits & 0xFFFFu), __NV_E4M3);
+  return h2bits(__half2(r));
+}
+
 constexpr int kGroupWarps = 8;                  // consumer warps sharing one head
 constexpr int kGroups = 2;                      // consumer groups, alternating items
 constexpr int kGroupThreads = kGroupWarps * 32;
@@ -247,7 +281,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   const int XOFF = TB + SB;
   const size_t stage_bytes = ((size_t)XOFF + (size_t)(L + MAXM) * XROW + 127) & ~(size_t)127;
   // each group's region starts on a 128-byte boundary (float4 reads of B and C rows)
-  const int group_floats = (WMAX * N + MAXM * N + hc * WMAX + MAXM * WMAX + hc * HS + 31) & ~31;
+  constexpr bool kMma = mma_read<P, N, Tin, RF, MAXM>();
+  constexpr int kUnitWarps = kMma ? 4 : kGroupWarps;   // warps that work on (and release) one head
+  const int mma_off = (WMAX * N + MAXM * N + hc * WMAX + MAXM * WMAX + hc * HS + 3) & ~3;
+  const int group_floats = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~31;
 
   const Tin *xin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *Bin = reinterpret_cast<const Tin *>(a.in[1]);
@@ -266,7 +303,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGroupWarps);
+      mbar_init(&empty[s], kUnitWarps);
       stage_use[s] = -1;
     }
     abort_flag = 0;
@@ -359,7 +396,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   float *sdt = sC + MAXM * N;                                          // [hc][WMAX]
   float *sBC = sdt + hc * WMAX;                                        // [MAXM][WMAX]
   float *ssc = sBC + MAXM * WMAX;                                      // [hc][HS]
-  const int row0 = gw * T::RPW + lane / T::LPR;
+  __half *sCh = reinterpret_cast<__half *>(sB + mma_off);              // [N] C as f16 (tensor-core path)
+  float *sCinv = sB + mma_off + N / 2;                                 // 1 / its power-of-two scale
+  const int sub = kMma ? (gw >> 2) : 0;   // tensor-core path: 4-warp half of the group, alternate heads
   const int c0 = (lane % T::LPR) * 4;
   for (int k = gi; k < my_items; k += kGroups) {
     int b, g, chunk;
@@ -419,6 +458,16 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         acc = warp_sum(acc);
         if (lane == 0) sBC[j * WMAX + i] = acc;
       }
+      if constexpr (kMma) {
+        if (gw == kGroupWarps - 1) {   // C as f16, scaled so that max |C| is in [2^14, 2^15)
+          float cm = 0.0f;
+          for (int c = lane; c < N; c += 32) cm = fmaxf(cm, fabsf(sC[c]));
+          cm = group_max<32>(cm);
+          const int e = cm > 0.0f ? 14 - ilogbf(cm) : 0;
+          for (int c = lane; c < N; c += 32) sCh[c] = __float2half_rn(ldexpf(sC[c], e));
+          if (lane == 0) *sCinv = ldexpf(1.0f, -e);
+        }
+      }
       named_sync(bar_id, kGroupThreads);
       // ---- window scalars of every head: per (head, task) one warp.  Output j:
       //      coef_ji = e^{A seg(i, e_j)} dt_i (B_i . C_j) for i in [w0, e_j] (0
@@ -474,15 +523,31 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
       return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
     };
+    constexpr int hstep = kMma ? 2 : 1;   // heads taken by this warp: sub, sub + hstep, ...
     {
-      const int seq = seq_base + (inter ? (k & 1) : (k & 1) * hc);   // the item's first head
+      const int seq = seq_base + (inter ? 2 * sub + (k & 1) : (k & 1) * hc + sub);   // its first head
       s = seq % stages;
       use = seq / stages;
     }
-    const int step = inter ? 2 : 1;
-    for (int jh = 0; jh < hc; ++jh, s += step) {
+    const int step = (inter ? 2 : 1) * hstep;
+    // tensor-core path: the B fragments (C as f16, column 0) for the item, in
+    // the permuted k order: thread (g, t) holds C[32 t + 4 ks .. + 3]
+    uint32_t bfr[kMma ? 16 : 1];
+    float cinv = 0.0f;
+    if constexpr (kMma) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint2 v = make_uint2(0u, 0u);
+        if ((lane >> 2) == 0 && !rp.refuse)
+          v = *reinterpret_cast<const uint2 *>(sCh + 32 * (lane & 3) + 4 * ks);
+        bfr[2 * ks] = v.x;
+        bfr[2 * ks + 1] = v.y;
+      }
+      if (!rp.refuse) cinv = *sCinv;
+    }
+    for (int jh = sub; jh < hc; jh += hstep, s += step) {
       const int h = h0 + jh;
-      if (s >= stages) {
+      while (s >= stages) {
         s -= stages;
         ++use;
       }
@@ -495,63 +560,137 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         const float *hs = ssc + jh * HS;
         const float *hcoef = hs, *hdec = hs + MAXM * 32, *hfw = hs + MAXM * 32 + MAXM;
         const float *hdecf = hfw + 64;
-        float4 f[T::NLD];   // fp32 checkpoint values for a fold (read-copy layers)
-        if constexpr (RF != RSSM_READ_FP32) {
-          if (pre || post) {
-#pragma unroll
-            for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_tile + (size_t)(row0 + l * T::RPI) * N + c0);
-          }
-        }
         if (!wait_stage()) break;
         const Stage stg{smem + s * stage_bytes, XOFF, XROW, n, L};
-
-        float4 v[T::NLD];
-        if (pre) {   // the new tokens do not fit: fold the committed window first
-          if constexpr (RF == RSSM_READ_FP32) {
+        bool done = false;
+        if constexpr (kMma) {
+          if (!pre && !post) {   // ---- tensor-core read: this warp's 16-row tile
+            const int mt = gw & 3, g8 = lane >> 2, t4 = lane & 3;
+            const int ra = mt * 16 + g8, rb = ra + 8;
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            uint32_t af[4];
+            if constexpr (RF == RSSM_READ_NVFP4) {
+              // thread t4 holds bytes [16 t4, 16 t4 + 16) of its rows: k-step ks uses
+              // bytes 2 ks (k pair t4) and 2 ks + 1 (k pair t4 + 4); scale block
+              // 2 t4 + ks / 4
+              const uint4 qa = *reinterpret_cast<const uint4 *>(stg.base + (size_t)ra * RB + 16 * t4);
+              const uint4 qb = *reinterpret_cast<const uint4 *>(stg.base + (size_t)rb * RB + 16 * t4);
+              const __half2 sa = __half2(__nv_cvt_fp8x2_to_halfraw2(
+                  *reinterpret_cast<const uint16_t *>(stg.base + TB + ra * (N / 16) + 2 * t4), __NV_E4M3));
+              const __half2 sbl = __half2(__nv_cvt_fp8x2_to_halfraw2(
+                  *reinterpret_cast<const uint16_t *>(stg.base + TB + rb * (N / 16) + 2 * t4), __NV_E4M3));
+              const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-            for (int l = 0; l < T::NLD; ++l)
-              f[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(row0 + l * T::RPI) * N + c0) * 4);
-          }
-          fold_tile<P, N, kGroupWarps, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
-#pragma unroll
-          for (int l = 0; l < T::NLD; ++l) {
-            const int row = row0 + l * T::RPI;
-            if (!post) st_stream(hc_tile + (size_t)row * N + c0, f[l]);
-            if constexpr (RF == RSSM_READ_FP32)
-              v[l] = f[l];
-            else
-              v[l] = quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
-          }
-        } else {
-#pragma unroll
-          for (int l = 0; l < T::NLD; ++l) {
-            const int row = row0 + l * T::RPI;
-            if constexpr (RF == RSSM_READ_FP32) {
-              v[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)row * N + c0) * 4);
-            } else if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
-              const uint32_t w = *reinterpret_cast<const uint32_t *>(stg.base + (size_t)row * RB + c0);
-              dec_e4m3x4(w, reinterpret_cast<const float *>(stg.base + TB)[row], v[l]);
+              for (int ks = 0; ks < 8; ++ks) {
+                const __half2 sca = ks < 4 ? __low2half2(sa) : __high2half2(sa);
+                const __half2 scb = ks < 4 ? __low2half2(sbl) : __high2half2(sbl);
+                const int sh = (ks & 1) * 16;
+                af[0] = e2m1x2_scaled(wa[ks >> 1] >> sh, sca);
+                af[1] = e2m1x2_scaled(wb[ks >> 1] >> sh, scb);
+                af[2] = e2m1x2_scaled(wa[ks >> 1] >> (sh + 8), sca);
+                af[3] = e2m1x2_scaled(wb[ks >> 1] >> (sh + 8), scb);
+                mma_16816(d, af, bfr[2 * ks], bfr[2 * ks + 1]);
+              }
             } else {
-              const uint32_t w = *reinterpret_cast<const uint16_t *>(stg.base + (size_t)row * RB + c0 / 2);
-              const float sc = dec_e4m3(stg.base[TB + row * (N / 16) + c0 / 16]);
-              dec_e2m1x4(w, sc, v[l]);
+              // thread t4 holds bytes [32 t4, 32 t4 + 32) of its rows: k-step ks uses the
+              // 4 bytes 4 ks .. 4 ks + 3 (k pairs t4 and t4 + 4); row scale after
+              const uint4 qa0 = *reinterpret_cast<const uint4 *>(stg.base + (size_t)ra * RB + 32 * t4);
+              const uint4 qa1 = *reinterpret_cast<const uint4 *>(stg.base + (size_t)ra * RB + 32 * t4 + 16);
+              const uint4 qb0 = *reinterpret_cast<const uint4 *>(stg.base + (size_t)rb * RB + 32 * t4);
+              const uint4 qb1 = *reinterpret_cast<const uint4 *>(stg.base + (size_t)rb * RB + 32 * t4 + 16);
+              const uint32_t wa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
+              const uint32_t wb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks) {
+                af[0] = e4m3x2_h2(wa[ks]);
+                af[1] = e4m3x2_h2(wb[ks]);
+                af[2] = e4m3x2_h2(wa[ks] >> 16);
+                af[3] = e4m3x2_h2(wb[ks] >> 16);
+                mma_16816(d, af, bfr[2 * ks], bfr[2 * ks + 1]);
+              }
+              const float *srow = reinterpret_cast<const float *>(stg.base + TB);
+              d[0] *= srow[ra];
+              d[2] *= srow[rb];
             }
+            // Epilogue: lane (r16 = lane & 15, entry parity lane >> 4) sums the window
+            // terms of row r16 over every other entry; the h C value of row r16 sits
+            // in d[0] (r16 < 8) or d[2] of lane 4 (r16 & 7).
+            const int r16 = lane & 15, row = mt * 16 + r16;
+            float ws = 0.0f;
+            for (int i = w0 + (lane >> 4); i <= n; i += 2) ws = fmaf(hcoef[i - w0], stg.x<Tin>(i, row), ws);
+            ws += __shfl_xor_sync(kFull, ws, 16);
+            const float va = __shfl_sync(kFull, d[0], 4 * (r16 & 7));
+            const float vb = __shfl_sync(kFull, d[2], 4 * (r16 & 7));
+            if (lane < 16) {
+              const float hcv = (r16 < 8 ? va : vb) * cinv;
+              a.out[((size_t)b * a.H + h) * P + row] =
+                  fmaf(__ldg(a.D + h), stg.x<Tin>(n, row), fmaf(hdec[0], hcv, ws));
+            }
+            done = true;
           }
         }
-        if (m > 0)
-          outputs<P, N, kGroupWarps, Tin, MAXM>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
-        if (post) {  // the decode filled the window: fold all of it
-          if constexpr (RF == RSSM_READ_FP32) {
+        if (!done) {
+          // ---- CUDA-core path, per group of 8 rows ("virtual warp"; two per warp
+          //      when four warps share a head)
+#pragma unroll 1
+          for (int vw = 0; vw < (kMma ? 2 : 1); ++vw) {
+            const int row0 = (kMma ? ((gw & 3) * 2 + vw) : gw) * T::RPW + lane / T::LPR;
+            float4 f[T::NLD];   // fp32 checkpoint values for a fold (read-copy layers)
+            if constexpr (RF != RSSM_READ_FP32) {
+              if (pre || post) {
 #pragma unroll
-            for (int l = 0; l < T::NLD; ++l) f[l] = v[l];
-          }
-          fold_tile<P, N, kGroupWarps, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
+                for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_tile + (size_t)(row0 + l * T::RPI) * N + c0);
+              }
+            }
+            float4 v[T::NLD];
+            if (pre) {   // the new tokens do not fit: fold the committed window first
+              if constexpr (RF == RSSM_READ_FP32) {
 #pragma unroll
-          for (int l = 0; l < T::NLD; ++l) {
-            const int row = row0 + l * T::RPI;
-            st_stream(hc_tile + (size_t)row * N + c0, f[l]);
-            if constexpr (RF != RSSM_READ_FP32)
-              quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+                for (int l = 0; l < T::NLD; ++l)
+                  f[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(row0 + l * T::RPI) * N + c0) * 4);
+              }
+              fold_tile<P, N, kGroupWarps, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
+#pragma unroll
+              for (int l = 0; l < T::NLD; ++l) {
+                const int row = row0 + l * T::RPI;
+                if (!post) st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+                if constexpr (RF == RSSM_READ_FP32)
+                  v[l] = f[l];
+                else
+                  v[l] = quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+              }
+            } else {
+#pragma unroll
+              for (int l = 0; l < T::NLD; ++l) {
+                const int row = row0 + l * T::RPI;
+                if constexpr (RF == RSSM_READ_FP32) {
+                  v[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)row * N + c0) * 4);
+                } else if constexpr (RF == RSSM_READ_FP8_E4M3_ROW) {
+                  const uint32_t w = *reinterpret_cast<const uint32_t *>(stg.base + (size_t)row * RB + c0);
+                  dec_e4m3x4(w, reinterpret_cast<const float *>(stg.base + TB)[row], v[l]);
+                } else {
+                  const uint32_t w = *reinterpret_cast<const uint16_t *>(stg.base + (size_t)row * RB + c0 / 2);
+                  const float sc = dec_e4m3(stg.base[TB + row * (N / 16) + c0 / 16]);
+                  dec_e2m1x4(w, sc, v[l]);
+                }
+              }
+            }
+            if (m > 0)
+              outputs<P, N, kGroupWarps, Tin, MAXM>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
+            if (post) {  // the decode filled the window: fold all of it
+              if constexpr (RF == RSSM_READ_FP32) {
+#pragma unroll
+                for (int l = 0; l < T::NLD; ++l) f[l] = v[l];
+              }
+              fold_tile<P, N, kGroupWarps, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
+#pragma unroll
+              for (int l = 0; l < T::NLD; ++l) {
+                const int row = row0 + l * T::RPI;
+                st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+                if constexpr (RF != RSSM_READ_FP32)
+                  quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+              }
+            }
           }
         }
       }
@@ -659,8 +798,9 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
   const size_t xrow = (size_t)P * sizeof(Tin);
   const size_t stage = ((size_t)tile_bytes<RF, P, N>() + scale_bytes<RF, P, N>() + (a.L + MAXM) * xrow + 127) & ~(size_t)127;
   const size_t wmax = a.L + MAXM;
-  const size_t group_floats = (wmax * N + MAXM * N + hc * wmax + MAXM * wmax +
-                               (size_t)hc * (MAXM * 32 + MAXM + 64 + 2) + 31) & ~(size_t)31;
+  const size_t mma_off = (wmax * N + MAXM * N + hc * wmax + MAXM * wmax +
+                          (size_t)hc * (MAXM * 32 + MAXM + 64 + 2) + 3) & ~(size_t)3;
+  const size_t group_floats = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~(size_t)31;
   const size_t fixed = kGroups * sizeof(float) * group_floats;
   // One CTA per SM (its 544 threads use the register file); as many stages as
   // fit in its shared memory, at most 5 for fp32 tiles (32 KiB each) and
