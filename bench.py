@@ -527,6 +527,45 @@ def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6):
     return res
 
 
+def quantized_state_leg(base, calls=96, warmup=16):
+    """The conventional step on a state stored in FP8 / NVFP4 and rounded again
+    every token (the design a read copy replaces): tokens/s and GB/s of state
+    and token bytes, same layer shape and tokens as `base`."""
+    import copy
+    from hybrid_ssm_decode_replayssm_b200 import rssm
+    res = {}
+    s = base.shape
+    rows, cols = (s.batch * s.nheads * (s.headdim if base.name == "mamba2" else s.dv),
+                  s.dstate if base.name == "mamba2" else s.dk)
+    for name, fmt in (("fp8_e4m3_row", rssm.RSSM_READ_FP8_E4M3_ROW), ("nvfp4", rssm.RSSM_READ_NVFP4)):
+        work = copy.copy(base)
+        work.desc = copy.copy(base.desc)
+        work.desc.read_fmt = fmt
+        layer = work.layer()
+        codes, scales = layer.quantized_state_buffers()
+        rc_codes, rc_scales = layer.read_copy_views()
+        codes.copy_(rc_codes)
+        scales.copy_(rc_scales)
+        out = torch.empty(work.out_shape, device=work.dev)
+        for t in range(warmup):
+            layer.conventional_step_quantized(codes, scales, codes, scales, work.pool[t % POOL], out)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record()
+        for t in range(calls):
+            layer.conventional_step_quantized(codes, scales, codes, scales, work.pool[t % POOL], out)
+        stop.record()
+        torch.cuda.synchronize()
+        el = start.elapsed_time(stop) / 1e3
+        state = codes.numel() + scales.numel() * scales.element_size()
+        tok_bytes = work.conventional_bytes() - 2 * rows * cols * 4    # inputs and outputs
+        res[name] = {"tokens_per_s": round(s.batch * calls / el, 1),
+                     "hbm_gbs": round((2 * state + tok_bytes) * calls / el / 1e9, 1)}
+        del layer, codes, scales
+        torch.cuda.empty_cache()
+    return res
+
+
 # -------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -539,7 +578,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
-    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy",
+    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -621,7 +660,7 @@ def main():
     if "e2e" in legs:
         del e2e_layer
     gw = None
-    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy"}:
+    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state"}:
         gw = GDNWork(dev, seed, args.batch)
     if world == 1 and "gdn" in legs and gw is not None:
         gl = gw.layer()
@@ -649,6 +688,12 @@ def main():
         extras["read_copy"] = {work.name: read_copy_leg(work)}
         if gw is not None:
             extras["read_copy"]["gdn"] = read_copy_leg(gw)
+    if world == 1 and "quantized_state" in legs:
+        extras["quantized_state_baseline"] = {
+            "how": "conventional step on a state stored in the format and rounded again every token",
+            work.name: quantized_state_leg(work)}
+        if gw is not None:
+            extras["quantized_state_baseline"]["gdn"] = quantized_state_leg(gw)
     del gw
     torch.cuda.empty_cache()
 

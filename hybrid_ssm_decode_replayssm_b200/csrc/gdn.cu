@@ -884,8 +884,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 
 // Conventional gated delta rule: per row i of S (16 warps x 8 rows, a lane owns
 // 4 columns): u_i = alpha S_i.k, o_i = out_scale (alpha S_i.q + c_i (k.q)),
-// S_i <- alpha S_i + c_i k with c_i = beta (v_i - u_i); S written back.
-template <typename Tin>
+// S_i <- alpha S_i + c_i k with c_i = beta (v_i - u_i); S written back.  SF
+// (state format): fp32, or a state kept in low precision (FP8 row / NVFP4,
+// read-copy layout), decoded, updated in fp32 and rounded again every token
+// (o comes from the updated fp32 values before that rounding).
+template <typename Tin, int SF>
 __global__ void __launch_bounds__(512) gdn_conv_kernel(const ConvArgs a) {
   constexpr int R8 = DV / 16;
   __shared__ float s_c[DV], s_kq;
@@ -894,10 +897,16 @@ __global__ void __launch_bounds__(512) gdn_conv_kernel(const ConvArgs a) {
   const int b = (int)(bh / a.H);
   (void)b;
   const int c0 = lane * 4, row0 = warp * R8;
-  const float *S = a.state_in + bh * DV * DK;
+  constexpr int RB = rc_row_bytes<SF>();
   float4 t[R8];
 #pragma unroll
-  for (int r = 0; r < R8; ++r) t[r] = ld_stream(S + (size_t)(row0 + r) * DK + c0);
+  for (int r = 0; r < R8; ++r) {
+    const size_t row = bh * DV + row0 + r;
+    if constexpr (SF == RSSM_READ_FP32)
+      t[r] = ld_stream(a.state_in + row * DK + c0);
+    else
+      t[r] = load_read_copy4<SF>(a.codes_in + row * RB, a.scales_in, row, DK, c0);
+  }
   const Tin *q = reinterpret_cast<const Tin *>(a.in[0]) + bh * DK;
   const Tin *k = reinterpret_cast<const Tin *>(a.in[1]) + bh * DK;
   const Tin *v = reinterpret_cast<const Tin *>(a.in[2]) + bh * DV;
@@ -934,7 +943,11 @@ __global__ void __launch_bounds__(512) gdn_conv_kernel(const ConvArgs a) {
   for (int r = 0; r < R8; ++r) {
     scale4(t[r], alpha);
     fma4(t[r], s_c[row0 + r], kc);
-    st_stream(a.state_out + bh * DV * DK + (size_t)(row0 + r) * DK + c0, t[r]);
+    const size_t row = bh * DV + row0 + r;
+    if constexpr (SF == RSSM_READ_FP32)
+      st_stream(a.state_out + row * DK + c0, t[r]);
+    else
+      quantize4<SF, 32>(t[r], a.codes_out + row * RB, a.scales_out, row, DK, c0, lane);
   }
 }
 
@@ -1000,6 +1013,15 @@ cudaError_t dispatch_rf(const StepArgs &a, int rf, cudaStream_t s) {
   }
 }
 
+template <int SF>
+cudaError_t launch_conv(const ConvArgs &a, int in_dtype, cudaStream_t s) {
+  if (in_dtype == RSSM_BF16)
+    gdn_conv_kernel<__nv_bfloat16, SF><<<dim3((unsigned)(a.B * a.H)), dim3(512), 0, s>>>(a);
+  else
+    gdn_conv_kernel<float, SF><<<dim3((unsigned)(a.B * a.H)), dim3(512), 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool gdn_supported(int R, int C) { return R == DV && C == DK; }
@@ -1009,12 +1031,12 @@ cudaError_t gdn_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t
   return dispatch_rf<float>(a, read_fmt, s);
 }
 
-cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s) {
-  if (in_dtype == RSSM_BF16)
-    gdn_conv_kernel<__nv_bfloat16><<<dim3((unsigned)(a.B * a.H)), dim3(512), 0, s>>>(a);
-  else
-    gdn_conv_kernel<float><<<dim3((unsigned)(a.B * a.H)), dim3(512), 0, s>>>(a);
-  return cudaGetLastError();
+cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s) {
+  switch (state_fmt) {
+    case RSSM_READ_FP32: return launch_conv<RSSM_READ_FP32>(a, in_dtype, s);
+    case RSSM_READ_FP8_E4M3_ROW: return launch_conv<RSSM_READ_FP8_E4M3_ROW>(a, in_dtype, s);
+    default: return launch_conv<RSSM_READ_NVFP4>(a, in_dtype, s);
+  }
 }
 
 }  // namespace rssm

@@ -734,7 +734,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 }
 
 // Conventional update: h <- e^{dt A} h + dt x B^T ; y = h C + D x ; h written back.
-template <int P, int N, typename Tin>
+// SF (state format): fp32, or a state kept in low precision (FP8 row / NVFP4,
+// read-copy layout) that is decoded, updated in fp32 and rounded again every
+// token; y comes from the updated fp32 values before that rounding.
+template <int P, int N, typename Tin, int SF>
 __global__ void __launch_bounds__(kThreads) m2_conv_kernel(const ConvArgs a) {
   using T = Tile<P, N>;
   __shared__ __align__(16) float s_x[P];
@@ -745,10 +748,16 @@ __global__ void __launch_bounds__(kThreads) m2_conv_kernel(const ConvArgs a) {
   const size_t bh = (size_t)b * a.H + h;
   const int row0 = warp * T::RPW + lane / T::LPR;
   const int c0 = (lane % T::LPR) * 4;
+  constexpr int RB = rc_row_bytes<SF, N>();
   float4 t[T::NLD];
 #pragma unroll
-  for (int l = 0; l < T::NLD; ++l)
-    t[l] = ld_stream(a.state_in + bh * P * N + (size_t)(row0 + l * T::RPI) * N + c0);
+  for (int l = 0; l < T::NLD; ++l) {
+    const size_t row = bh * P + row0 + l * T::RPI;
+    if constexpr (SF == RSSM_READ_FP32)
+      t[l] = ld_stream(a.state_in + row * N + c0);
+    else
+      t[l] = load_read_copy4<SF>(a.codes_in + row * RB, a.scales_in, row, N, c0);
+  }
   const Tin *xin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *Bin = reinterpret_cast<const Tin *>(a.in[1]);
   const Tin *Cin = reinterpret_cast<const Tin *>(a.in[2]);
@@ -770,7 +779,10 @@ __global__ void __launch_bounds__(kThreads) m2_conv_kernel(const ConvArgs a) {
     t[l].y = fmaf(xr, bv.y, dA * t[l].y);
     t[l].z = fmaf(xr, bv.z, dA * t[l].z);
     t[l].w = fmaf(xr, bv.w, dA * t[l].w);
-    st_stream(a.state_out + bh * P * N + (size_t)row * N + c0, t[l]);
+    if constexpr (SF == RSSM_READ_FP32)
+      st_stream(a.state_out + bh * P * N + (size_t)row * N + c0, t[l]);
+    else
+      quantize4<SF, T::LPR>(t[l], a.codes_out + (bh * P + row) * RB, a.scales_out, bh * P + row, N, c0, lane);
     part[l] = t[l].x * cv.x + t[l].y * cv.y + t[l].z * cv.z + t[l].w * cv.w;
   }
   tr_sum<T::NLD, T::LPR / 2>(part, lane);
@@ -849,13 +861,22 @@ cudaError_t dispatch_dtype(const StepArgs &a, int in_dtype, int rf, cudaStream_t
   return dispatch_rf<P, N, float>(a, rf, s);
 }
 
-template <int P, int N>
-cudaError_t launch_conv(const ConvArgs &a, int in_dtype, cudaStream_t s) {
+template <int P, int N, int SF>
+cudaError_t launch_conv_fmt(const ConvArgs &a, int in_dtype, cudaStream_t s) {
   if (in_dtype == RSSM_BF16)
-    m2_conv_kernel<P, N, __nv_bfloat16><<<dim3((unsigned)(a.B * a.H)), dim3(kThreads), 0, s>>>(a);
+    m2_conv_kernel<P, N, __nv_bfloat16, SF><<<dim3((unsigned)(a.B * a.H)), dim3(kThreads), 0, s>>>(a);
   else
-    m2_conv_kernel<P, N, float><<<dim3((unsigned)(a.B * a.H)), dim3(kThreads), 0, s>>>(a);
+    m2_conv_kernel<P, N, float, SF><<<dim3((unsigned)(a.B * a.H)), dim3(kThreads), 0, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int P, int N>
+cudaError_t launch_conv(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s) {
+  switch (state_fmt) {
+    case RSSM_READ_FP32: return launch_conv_fmt<P, N, RSSM_READ_FP32>(a, in_dtype, s);
+    case RSSM_READ_FP8_E4M3_ROW: return launch_conv_fmt<P, N, RSSM_READ_FP8_E4M3_ROW>(a, in_dtype, s);
+    default: return launch_conv_fmt<P, N, RSSM_READ_NVFP4>(a, in_dtype, s);
+  }
 }
 
 }  // namespace
@@ -867,9 +888,9 @@ cudaError_t mamba2_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStrea
   return dispatch_dtype<64, 128>(a, in_dtype, read_fmt, s);
 }
 
-cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s) {
-  if (a.R == 64 && a.C == 64) return launch_conv<64, 64>(a, in_dtype, s);
-  return launch_conv<64, 128>(a, in_dtype, s);
+cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s) {
+  if (a.R == 64 && a.C == 64) return launch_conv<64, 64>(a, in_dtype, state_fmt, s);
+  return launch_conv<64, 128>(a, in_dtype, state_fmt, s);
 }
 
 }  // namespace rssm

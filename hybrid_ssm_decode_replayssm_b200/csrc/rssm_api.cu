@@ -307,10 +307,47 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev, float *sta
   a.state_in = state_in_dev; a.state_out = state_out_dev;
   for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
   a.out = static_cast<float *>(out_dev);
-  cudaError_t e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_conventional(a, h->d.in_dtype, (cudaStream_t)stream)
-                                           : rssm::gdn_conventional(a, h->d.in_dtype, (cudaStream_t)stream);
+  cudaError_t e = h->d.kind == RSSM_MAMBA2
+                      ? rssm::mamba2_conventional(a, h->d.in_dtype, RSSM_READ_FP32, (cudaStream_t)stream)
+                      : rssm::gdn_conventional(a, h->d.in_dtype, RSSM_READ_FP32, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "conventional kernel launch");
+  return ok();
+}
+
+int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev, const void *scales_in_dev,
+                                     void *codes_out_dev, void *scales_out_dev, const void *const *in,
+                                     void *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.read_fmt == RSSM_READ_FP32)
+    return fail(RSSM_ERR_STATE, "the layer has no low-precision format (read_fmt is RSSM_READ_FP32)");
+  if (!codes_in_dev || !scales_in_dev || !codes_out_dev || !scales_out_dev)
+    return fail(RSSM_ERR_INVALID_ARG, "state code and scale pointers must not be NULL");
+  if (!aligned(codes_in_dev, 16) || !aligned(codes_out_dev, 16))
+    return fail(RSSM_ERR_INVALID_ARG, "state code pointers must be 16-byte aligned");
+  if (h->d.read_fmt == RSSM_READ_FP8_E4M3_ROW && (!aligned(scales_in_dev, 4) || !aligned(scales_out_dev, 4)))
+    return fail(RSSM_ERR_INVALID_ARG, "FP8 row scales must be 4-byte aligned");
+  int rc = check_inputs(h, in, out_dev);
+  if (rc) return rc;
+  rssm::ConvArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.B = h->d.batch; a.H = h->d.nheads;
+  a.G = h->d.kind == RSSM_MAMBA2 ? h->d.ngroups : 1;
+  a.hpg = a.H / a.G;
+  a.R = h->d.headdim; a.C = h->d.dstate;
+  a.out_scale = h->d.out_scale;
+  a.A = h->A; a.D = h->D;
+  a.codes_in = static_cast<const uint8_t *>(codes_in_dev);
+  a.scales_in = scales_in_dev;
+  a.codes_out = static_cast<uint8_t *>(codes_out_dev);
+  a.scales_out = scales_out_dev;
+  for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
+  a.out = static_cast<float *>(out_dev);
+  cudaError_t e = h->d.kind == RSSM_MAMBA2
+                      ? rssm::mamba2_conventional(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream)
+                      : rssm::gdn_conventional(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "quantized-state conventional kernel launch");
   return ok();
 }
 

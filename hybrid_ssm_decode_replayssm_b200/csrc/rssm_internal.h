@@ -47,8 +47,12 @@ struct ConvArgs {
   int B, H, G, hpg, R, C;
   float out_scale;
   const float *A, *D;
-  const float *state_in;
+  const float *state_in;       // fp32 state (state format RSSM_READ_FP32)
   float *state_out;
+  const uint8_t *codes_in;     // low-precision state (FP8 row / NVFP4), read-copy layout
+  const void *scales_in;
+  uint8_t *codes_out;
+  void *scales_out;
   const void *in[5];
   float *out;
 };
@@ -63,9 +67,11 @@ struct QuantArgs {
 
 // Launchers return cudaGetLastError() of their launch.
 cudaError_t mamba2_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
-cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s);
+// state_fmt: RSSM_READ_FP32 (fp32 state), or the FP8 row / NVFP4 format of a
+// state stored in low precision and rounded again after every token
+cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s);
 cudaError_t gdn_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
-cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s);
+cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s);
 cudaError_t quantize_read_copy(const QuantArgs &a, int read_fmt, cudaStream_t s);
 cudaError_t rollback(int B, const int32_t *n_reject, int32_t *len, int32_t *pending,
                      uint32_t *status, cudaStream_t s);

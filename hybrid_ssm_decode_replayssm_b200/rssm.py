@@ -32,7 +32,7 @@ EXPORTED = [
     "rssm_decode_step", "rssm_verify", "rssm_rollback", "rssm_flush",
     "rssm_quantize_read_copy", "rssm_conventional_step", "rssm_get_bookkeeping",
     "rssm_get_status", "rssm_last_error_string", "rssm_launch_count",
-    "rssm_decode_step_static_scratch",
+    "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -77,6 +77,7 @@ def lib():
         L.rssm_flush.argtypes = [vp, vp, vp]
         L.rssm_quantize_read_copy.argtypes = [vp, vp]
         L.rssm_conventional_step.argtypes = [vp, vp, vp, C.POINTER(vp), vp, vp]
+        L.rssm_conventional_step_quantized.argtypes = [vp, vp, vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_get_bookkeeping.argtypes = [vp, vp, vp]
         L.rssm_get_status.argtypes = [vp, C.POINTER(C.c_uint32), i32, vp]
         for name in EXPORTED:
@@ -190,6 +191,29 @@ class ReplayLayer:
         check(lib().rssm_conventional_step(self.handle, state_in.data_ptr(), state_out.data_ptr(),
                                            _ptr_array(inputs), out.data_ptr(), _stream(stream)))
         return out
+
+    def conventional_step_quantized(self, codes_in, scales_in, codes_out, scales_out, inputs, out,
+                                    stream=None):
+        """One conventional token on a state kept in the layer's low-precision format
+        (buffers from quantized_state_buffers(); in and out may be the same)."""
+        check(lib().rssm_conventional_step_quantized(
+            self.handle, codes_in.data_ptr(), scales_in.data_ptr(), codes_out.data_ptr(),
+            scales_out.data_ptr(), _ptr_array(inputs), out.data_ptr(), _stream(stream)))
+        return out
+
+    def quantized_state_buffers(self):
+        """(codes uint8, scales) tensors for a state stored in the layer's read format,
+        shaped as read_copy_views()."""
+        d = self.desc
+        B, H, R, Cc = d.batch, d.nheads, d.headdim, d.dstate
+        dev = self.ckpt.device
+        if d.read_fmt == RSSM_READ_FP8_E4M3_ROW:
+            return (torch.zeros((B, H, R, Cc), dtype=torch.uint8, device=dev),
+                    torch.zeros((B, H, R), dtype=torch.float32, device=dev))
+        if d.read_fmt == RSSM_READ_NVFP4:
+            return (torch.zeros((B, H, R, Cc // 2), dtype=torch.uint8, device=dev),
+                    torch.zeros((B, H, R, Cc // 16), dtype=torch.uint8, device=dev))
+        raise ValueError("layer has no low-precision format")
 
     def get_bookkeeping(self, stream=None) -> torch.Tensor:
         out = torch.empty((4, self.desc.batch), dtype=torch.int32, device=self.ckpt.device)

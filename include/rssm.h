@@ -230,6 +230,30 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev,
                            void *out_dev, rssm_stream_t stream);
 
 /*
+ * The conventional per-token update with the state itself kept in low
+ * precision -- the design a read copy replaces [summary ¶4: rounding a stored
+ * state again at every token compounds the error, while a read copy beside an
+ * fp32 recurrence does not].  A baseline for that comparison.
+ *
+ * The state is stored in the handle's read_fmt (RSSM_READ_FP8_E4M3_ROW or
+ * RSSM_READ_NVFP4), in the read-copy layout above: codes_in_dev/scales_in_dev
+ * hold it before the token, codes_out_dev/scales_out_dev receive it after (the
+ * same buffers may be passed for an in-place update).  Per token: decode the
+ * codes, apply the conventional update in fp32 (inputs as rssm_decode_step),
+ * write the output from the updated fp32 values, then quantise the updated
+ * state exactly as rssm_quantize_read_copy does and store it.  Uses only the
+ * handle's shape, formats and parameters; its checkpoint, read copy and
+ * window are untouched.
+ * Errors: RSSM_ERR_STATE if read_fmt is RSSM_READ_FP32; RSSM_ERR_INVALID_ARG
+ * for NULL or misaligned pointers (codes 16-byte, FP8 scales 4-byte aligned).
+ */
+int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev,
+                                     const void *scales_in_dev,
+                                     void *codes_out_dev, void *scales_out_dev,
+                                     const void *const *in, void *out_dev,
+                                     rssm_stream_t stream);
+
+/*
  * rssm_decode_step without any caller-provided scratch.  (This entry point has
  * no counterpart on the pages; it serves integration needs only.)
  *

@@ -51,7 +51,13 @@ Modules and what pins each one (tests marked ``not gpu``):
                   the committed state, committed state advanced by the accepted
                   prefix.  Pinned by the rollback invariant (equal to decoding
                   only the accepted tokens from scratch).
+* ``quantized_state`` the baseline a read copy replaces: the conventional
+                  update on a state stored in FP8/NVFP4 and rounded again every
+                  token [summary ¶4].  Pinned by exactly representable states
+                  being fixed points of a do-nothing token, by the output being
+                  the one of the state before rounding, and by its drift over
+                  many tokens exceeding one rounding of the exact state.
 
 No function here is "parity unpinned".
 """
-from . import bookkeeping, codecs, gdn, mamba2, replay, speculative  # noqa: F401
+from . import bookkeeping, codecs, gdn, mamba2, quantized_state, replay, speculative  # noqa: F401

@@ -112,6 +112,8 @@ def test_create_checks_pointers_and_enqueues_nothing():
         assert L.rssm_rollback(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
         assert L.rssm_quantize_read_copy(h, None) == rssm.RSSM_ERR_STATE
         assert L.rssm_conventional_step(h, None, fake, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+        # an fp32-read layer has no low-precision state format
+        assert L.rssm_conventional_step_quantized(h, fake, fake, fake, fake, ins, fake, None) == rssm.RSSM_ERR_STATE
         assert L.rssm_get_bookkeeping(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
         assert L.rssm_get_status(h, None, 0, None) == rssm.RSSM_ERR_INVALID_ARG
     finally:
@@ -121,6 +123,29 @@ def test_create_checks_pointers_and_enqueues_nothing():
     L.rssm_set_params(h, fake, fake)
     assert L.rssm_verify(h, 1, ins, fake, None) == rssm.RSSM_ERR_STATE
     L.rssm_destroy(h)
+
+
+def test_quantized_state_step_checks_pointers():
+    L = rssm.lib()
+    fake = 1 << 20
+    for fmt in (rssm.RSSM_READ_FP8_E4M3_ROW, rssm.RSSM_READ_NVFP4):
+        d = _desc(read_fmt=fmt)
+        h = C.c_void_p()
+        assert L.rssm_create(C.byref(d), fake, fake, fake, fake, C.byref(h)) == rssm.RSSM_OK
+        try:
+            assert L.rssm_set_params(h, fake, fake) == rssm.RSSM_OK
+            ins = (C.c_void_p * 4)(fake, fake, fake, fake)
+            q = L.rssm_conventional_step_quantized
+            assert q(h, None, fake, fake, fake, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+            assert q(h, fake, fake, fake, None, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+            assert q(h, fake + 8, fake, fake, fake, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+            if fmt == rssm.RSSM_READ_FP8_E4M3_ROW:   # fp32 row scales: 4-byte aligned
+                assert q(h, fake, fake + 2, fake, fake, ins, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+            assert q(h, fake, fake, fake, fake, ins, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        finally:
+            assert L.rssm_destroy(h) == rssm.RSSM_OK
+    assert L.rssm_conventional_step_quantized(None, None, None, None, None, None, None, None) == \
+        rssm.RSSM_ERR_INVALID_ARG
 
 
 def test_null_handle_everywhere():
