@@ -566,6 +566,47 @@ def quantized_state_leg(base, calls=96, warmup=16):
     return res
 
 
+def graph_leg(m2, gw, steps=48, warmup=16):
+    """A decode step of three layers (two Mamba-2 and one GDN layer of the serving
+    shapes) launched eagerly and replayed from one captured CUDA graph."""
+    layers = [m2.layer(), m2.layer(), gw.layer()]
+    works = [m2, m2, gw]
+    outs = [torch.empty(w.out_shape, device=w.dev) for w in works]
+    ins = [[t.clone() for t in w.pool[0]] for w in works]
+
+    def step():
+        for layer, i, o in zip(layers, ins, outs):
+            layer.decode_step(i, o)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    stop.record()
+    torch.cuda.synchronize()
+    eager = start.elapsed_time(stop) / 1e3 / steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        step()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        g.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    graphed = start.elapsed_time(stop) / 1e3 / steps
+    del g, layers
+    torch.cuda.empty_cache()
+    return {"layers": "2 x " + m2.workload.split(":")[0] + " + 1 x " + gw.workload.split(":")[0] + " (serving shapes)",
+            "eager_us_per_step": round(eager * 1e6, 1), "graph_us_per_step": round(graphed * 1e6, 1),
+            "graph_tokens_per_s": round(m2.shape.batch / graphed, 1)}
+
+
 # -------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -578,7 +619,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
-    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state",
+    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state,graph",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -660,7 +701,7 @@ def main():
     if "e2e" in legs:
         del e2e_layer
     gw = None
-    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state"}:
+    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state", "graph"}:
         gw = GDNWork(dev, seed, args.batch)
     if world == 1 and "gdn" in legs and gw is not None:
         gl = gw.layer()
@@ -688,6 +729,8 @@ def main():
         extras["read_copy"] = {work.name: read_copy_leg(work)}
         if gw is not None:
             extras["read_copy"]["gdn"] = read_copy_leg(gw)
+    if world == 1 and "graph" in legs and gw is not None:
+        extras["multi_layer_graph"] = graph_leg(work, gw)
     if world == 1 and "quantized_state" in legs:
         extras["quantized_state_baseline"] = {
             "how": "conventional step on a state stored in the format and rounded again every token",
