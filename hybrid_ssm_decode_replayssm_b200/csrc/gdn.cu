@@ -23,16 +23,17 @@
 // checkpoint (UT transform) and the copy's rounding never enters the state.
 //
 // Work unit: half a head (64 of the 128 value rows, 32 KiB of fp32 state).  A
-// persistent CTA has one producer warp, which streams units into a ring of
+// persistent CTA has one producer warp, which streams units into rings of
 // shared-memory stages with 1-D TMA bulk copies (the read tile and the cached
 // w rows; fold units of re-solving layers also the v rows), and two consumer
 // groups of 8 warps taking alternate items (item = one sequence and a chunk of
-// heads), whose units the producer interleaves (IssueOrder).  An item's
-// prologue copies the committed window k rows of its heads into shared memory
-// (cp.async), loads the gates, converts the new q, k, v rows to fp32, appends
-// to the ring and computes every head's window scalars.  Per unit each warp owns 8 state rows; a row is spread over 8
-// lanes (4 chunks of 4 columns each), so its dot products reduce in three
-// shuffle steps.
+// heads).  Each group has its own ring; the producer serves whichever group
+// has a free stage, so one group's item prologue overlaps the other's stream.
+// An item's prologue copies the committed window k rows of its heads into
+// shared memory (cp.async), loads the gates, converts the new q, k, v rows to
+// fp32, appends to the ring and computes every head's window scalars.  Per
+// unit each warp owns 8 state rows; a row is spread over 8 lanes (4 chunks of
+// 4 columns each), so its dot products reduce in three shuffle steps.
 #include "rssm_device.cuh"
 
 namespace rssm {
@@ -190,7 +191,6 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   constexpr int HSO = MAXM + 2 * MAXM * kMaxW;   // per head: dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
-  __shared__ int stage_use[kMaxStages];   // see the Mamba-2 kernel: gates parity waits
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -199,7 +199,6 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   const int nchunk = a.H / hc;
   const int nitems = a.B * nchunk;
   const int my_items = (int)blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  const int total_seq = my_items * hc * 2;
 
   const Tin *qin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *kin = reinterpret_cast<const Tin *>(a.in[1]);
@@ -215,7 +214,6 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kGroupWarps);
-      stage_use[s] = -1;
     }
     abort_flag = 0;
     mbar_fence_init();
@@ -231,35 +229,58 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    // Issue order: the units of items 2p and 2p + 1 alternate (see IssueOrder).
-    const IssueOrder<true> order(my_items, 2 * hc);
-    // the current item of each group (scalars, not arrays: no local memory)
+    // Each consumer group has its own ring of SPG = stages / 2 stages (group g:
+    // stages g SPG .. g SPG + SPG - 1) and consumes its units in order: unit t of
+    // group g (its item t / 2hc, unit t mod 2hc) uses stage g SPG + t mod SPG for
+    // the (t / SPG)-th time.  The producer serves whichever group has a free
+    // stage, so a group busy in its item prologue holds back only its own ring
+    // while the other group's stream goes on.
+    const int SPG = stages / 2;
+    const int T0 = ((my_items + 1) / 2) * 2 * hc, T1 = (my_items / 2) * 2 * hc;
+    int t0 = 0, t1 = 0, pref = 0;
     int b_0 = 0, b_1 = 0, chunk_0 = 0, chunk_1 = 0, cur_0 = -1, cur_1 = -1;
     RowPlan rp_0{}, rp_1{};
-    int s = 0, u = 0;
-    int issued = 0;
-    for (int seq = 0; seq < total_seq; ++seq) {
-      if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
-        atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
-        break;
+    long long idle_since = clock64();
+    bool timed_out = false;
+    while (t0 < T0 || t1 < T1) {
+      // the group to serve: the preferred one if its next stage is free, else the other
+      int g = -1;
+      for (int q = 0; q < 2 && g < 0; ++q) {
+        const int c = pref ^ q;
+        const int t = c ? t1 : t0;
+        if (t >= (c ? T1 : T0)) continue;
+        const int s_ = c * SPG + t % SPG, u_ = t / SPG;
+        if (u_ == 0 || mbar_try_wait(&empty[s_], (uint32_t)((u_ - 1) & 1))) g = c;
       }
-      int kc, unit;
-      order.unit_at(seq, kc, unit);
-      if (kc & 1) {
+      if (g < 0) {
+        if (*abort || clock64() - idle_since > 2000000000LL) {
+          timed_out = true;
+          break;
+        }
+        continue;
+      }
+      idle_since = clock64();
+      pref = g ^ 1;   // alternate when both can go
+      const int t = g ? t1 : t0;
+      const int s = g * SPG + t % SPG;
+      const int kk = t / (2 * hc), unit = t - kk * 2 * hc, kc = 2 * kk + g;
+      if (g) {
+        ++t1;
         if (kc != cur_1) {
           cur_1 = kc;
           item_of(kc, b_1, chunk_1);
           rp_1 = plan_row(a, b_1);
         }
-      } else if (kc != cur_0) {
-        cur_0 = kc;
-        item_of(kc, b_0, chunk_0);
-        rp_0 = plan_row(a, b_0);
+      } else {
+        ++t0;
+        if (kc != cur_0) {
+          cur_0 = kc;
+          item_of(kc, b_0, chunk_0);
+          rp_0 = plan_row(a, b_0);
+        }
       }
-      const bool g1 = kc & 1;
-      const int b = g1 ? b_1 : b_0, chunk = g1 ? chunk_1 : chunk_0;
-      const RowPlan rp = g1 ? rp_1 : rp_0;
-      issued = seq + 1;
+      const int b = g ? b_1 : b_0, chunk = g ? chunk_1 : chunk_0;
+      const RowPlan rp = g ? rp_1 : rp_0;
       if (rp.refuse) {
         mbar_arrive(&full[s]);
       } else {
@@ -297,15 +318,17 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           bulk_g2s(dst + Y.voff + (L + j) * VHROW, vin + tok * DV + hf * HALF, VHROW, &full[s]);
         }
       }
-      *reinterpret_cast<volatile int *>(&stage_use[s]) = u;
-      if (++s == stages) {
-        s = 0;
-        ++u;
-      }
     }
-    if (*abort) {
-      for (int q = issued - stages > 0 ? issued - stages : 0; q < issued; ++q)
-        mbar_wait_bounded(&full[q % stages], (uint32_t)((q / stages) & 1), nullptr, 200000000LL);
+    if (timed_out) {
+      *abort = 1;
+      atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
+    }
+    if (*abort) {   // let the copies requested on every stage land (bounded) before the CTA retires
+      for (int c = 0; c < 2; ++c) {
+        const int t = c ? t1 : t0;
+        for (int q = t - SPG > 0 ? t - SPG : 0; q < t; ++q)
+          mbar_wait_bounded(&full[c * SPG + q % SPG], (uint32_t)((q / SPG) & 1), nullptr, 200000000LL);
+      }
     }
     return;
   }
@@ -470,19 +493,16 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       }
     }
 
-    // stage and use of unit 2 jh + hf of this item, from its position in the
-    // producer's issue order
-    const IssueOrder<true> order(my_items, 2 * hc);
+    // stage and use of unit 2 jh + hf of this item in the group's own ring (the
+    // group's units in order: t = (k / 2) 2hc + 2 jh + hf)
+    const int SPG = stages / 2;
     int s = 0, use = 0;
     auto locate = [&](int jh, int hf) {
-      const int seq = order.seq(gi, k >> 1, 2 * jh + hf);
-      s = seq % stages;
-      use = seq / stages;
+      const int t = (k >> 1) * 2 * hc + 2 * jh + hf;
+      s = gi * SPG + t % SPG;
+      use = t / SPG;
     };
-    auto wait_stage = [&]() -> bool {
-      if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
-      return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
-    };
+    auto wait_stage = [&]() -> bool { return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort); };
     auto release_stage = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -971,11 +991,12 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
     if (a.H % c) continue;
     const Layout y = make_layout<Tin, RF, MAXM>(a.L, c);
     const size_t fixed = (size_t)kGroups * sizeof(float) * y.group_floats;
-    if (fixed + 2 * (size_t)y.stage_bytes > budget) continue;
+    if (fixed + 2 * (size_t)y.stage_bytes > budget) continue;   // at least one stage per group
     int st = (int)((budget - fixed) / y.stage_bytes);
     if (st > kMaxStages) st = kMaxStages;
     const long long items = (long long)a.B * (a.H / c);
     double cost = (double)((items + sms - 1) / sms) * (2 * c + 4);
+    st &= ~1;
     if (st < 4) cost *= 4.0 / st;
     if (hc == 0 || cost < best_cost) {
       hc = c;
@@ -984,6 +1005,7 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
     }
   }
   if (hc == 0) return cudaErrorInvalidConfiguration;
+  stages &= ~1;   // a ring of stages / 2 per consumer group
   const Layout y = make_layout<Tin, RF, MAXM>(a.L, hc);
   const size_t smem = (size_t)kGroups * sizeof(float) * y.group_floats + (size_t)stages * y.stage_bytes;
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;

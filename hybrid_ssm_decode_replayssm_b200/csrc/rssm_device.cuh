@@ -207,43 +207,6 @@ __device__ __forceinline__ float4 load_read_copy4(const uint8_t *codes_row, cons
   return out;
 }
 
-// ------------------------------------------------------------ issue order
-// Order in which the producer of a persistent replay CTA with two consumer
-// groups issues the units of its items.  Item k goes to group k % 2 as its
-// item k / 2; an item has `upi` units.
-//  * sequential: item after item (all of item 0, all of item 1, ...): the ring
-//    holds one group's units while the other group runs its item prologue.
-//  * interleaved: the units of items 2p and 2p + 1 alternate (a last unpaired
-//    item runs alone): both groups compute at once.
-// Mixing the groups' units with an offset was measured slower than either:
-// the units of a group busy in its prologue block the ring for the other.
-template <bool kInterleave>
-struct IssueOrder {
-  int my_items, upi;
-  __device__ IssueOrder(int items, int units) : my_items(items), upi(units) {}
-  // consumers: position of unit u of the group's item kk (CTA item 2 kk + g)
-  __device__ __forceinline__ int seq(int g, int kk, int u) const {
-    if constexpr (kInterleave) {
-      const bool paired = 2 * kk + 1 < my_items;
-      return kk * 2 * upi + (paired ? 2 * u + g : u);
-    } else {
-      return (2 * kk + g) * upi + u;
-    }
-  }
-  // producer: the CTA item and its unit at position `seq`
-  __device__ __forceinline__ void unit_at(int seq, int &k, int &u) const {
-    if constexpr (kInterleave) {
-      const int p = seq / (2 * upi), within = seq - p * 2 * upi;
-      const bool paired = 2 * p + 1 < my_items;
-      k = 2 * p + (paired ? (within & 1) : 0);
-      u = paired ? (within >> 1) : within;
-    } else {
-      k = seq / upi;
-      u = seq - k * upi;
-    }
-  }
-};
-
 // ------------------------------------------------- TMA bulk copies + mbarrier
 // 1-D bulk copies (cp.async.bulk, no tensor map, no multicast) from global to
 // this CTA's shared memory, completing on an mbarrier with a transaction count.
