@@ -229,13 +229,13 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    // Each consumer group has its own ring of SPG = stages / 2 stages (group g:
-    // stages g SPG .. g SPG + SPG - 1) and consumes its units in order: unit t of
-    // group g (its item t / 2hc, unit t mod 2hc) uses stage g SPG + t mod SPG for
-    // the (t / SPG)-th time.  The producer serves whichever group has a free
-    // stage, so a group busy in its item prologue holds back only its own ring
-    // while the other group's stream goes on.
-    const int SPG = stages / 2;
+    // Each consumer group has its own ring (group 0: stages 0 .. R0 - 1, group 1:
+    // stages R0 .. stages - 1; R0 = ceil(stages / 2)) and consumes its units in
+    // order: unit t of group g (its item t / 2hc, unit t mod 2hc) uses stage
+    // base_g + t mod R_g for the (t / R_g)-th time.  The producer serves
+    // whichever group has a free stage, so a group busy in its item prologue
+    // holds back only its own ring while the other group's stream goes on.
+    const int R0 = (stages + 1) / 2, R1 = stages - R0;
     const int T0 = ((my_items + 1) / 2) * 2 * hc, T1 = (my_items / 2) * 2 * hc;
     int t0 = 0, t1 = 0, pref = 0;
     int b_0 = 0, b_1 = 0, chunk_0 = 0, chunk_1 = 0, cur_0 = -1, cur_1 = -1;
@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         const int c = pref ^ q;
         const int t = c ? t1 : t0;
         if (t >= (c ? T1 : T0)) continue;
-        const int s_ = c * SPG + t % SPG, u_ = t / SPG;
+        const int Rc = c ? R1 : R0;
+        const int s_ = (c ? R0 : 0) + t % Rc, u_ = t / Rc;
         if (u_ == 0 || mbar_try_wait(&empty[s_], (uint32_t)((u_ - 1) & 1))) g = c;
       }
       if (g < 0) {
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       idle_since = clock64();
       pref = g ^ 1;   // alternate when both can go
       const int t = g ? t1 : t0;
-      const int s = g * SPG + t % SPG;
+      const int s = (g ? R0 : 0) + t % (g ? R1 : R0);
       const int kk = t / (2 * hc), unit = t - kk * 2 * hc, kc = 2 * kk + g;
       if (g) {
         ++t1;
@@ -325,9 +326,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     }
     if (*abort) {   // let the copies requested on every stage land (bounded) before the CTA retires
       for (int c = 0; c < 2; ++c) {
-        const int t = c ? t1 : t0;
-        for (int q = t - SPG > 0 ? t - SPG : 0; q < t; ++q)
-          mbar_wait_bounded(&full[c * SPG + q % SPG], (uint32_t)((q / SPG) & 1), nullptr, 200000000LL);
+        const int t = c ? t1 : t0, Rc = c ? R1 : R0;
+        for (int q = t - Rc > 0 ? t - Rc : 0; q < t; ++q)
+          mbar_wait_bounded(&full[(c ? R0 : 0) + q % Rc], (uint32_t)((q / Rc) & 1), nullptr, 200000000LL);
       }
     }
     return;
@@ -495,12 +496,12 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 
     // stage and use of unit 2 jh + hf of this item in the group's own ring (the
     // group's units in order: t = (k / 2) 2hc + 2 jh + hf)
-    const int SPG = stages / 2;
+    const int R0 = (stages + 1) / 2, Rg = gi ? stages - R0 : R0, base = gi ? R0 : 0;
     int s = 0, use = 0;
     auto locate = [&](int jh, int hf) {
       const int t = (k >> 1) * 2 * hc + 2 * jh + hf;
-      s = gi * SPG + t % SPG;
-      use = t / SPG;
+      s = base + t % Rg;
+      use = t / Rg;
     };
     auto wait_stage = [&]() -> bool { return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort); };
     auto release_stage = [&]() {
@@ -991,12 +992,11 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
     if (a.H % c) continue;
     const Layout y = make_layout<Tin, RF, MAXM>(a.L, c);
     const size_t fixed = (size_t)kGroups * sizeof(float) * y.group_floats;
-    if (fixed + 2 * (size_t)y.stage_bytes > budget) continue;   // at least one stage per group
+    if (fixed + 2 * (size_t)y.stage_bytes > budget) continue;   // at least one stage per group ring
     int st = (int)((budget - fixed) / y.stage_bytes);
     if (st > kMaxStages) st = kMaxStages;
     const long long items = (long long)a.B * (a.H / c);
     double cost = (double)((items + sms - 1) / sms) * (2 * c + 4);
-    st &= ~1;
     if (st < 4) cost *= 4.0 / st;
     if (hc == 0 || cost < best_cost) {
       hc = c;
@@ -1005,7 +1005,6 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
     }
   }
   if (hc == 0) return cudaErrorInvalidConfiguration;
-  stages &= ~1;   // a ring of stages / 2 per consumer group
   const Layout y = make_layout<Tin, RF, MAXM>(a.L, hc);
   const size_t smem = (size_t)kGroups * sizeof(float) * y.group_floats + (size_t)stages * y.stage_bytes;
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
