@@ -58,6 +58,14 @@ Modules and what pins each one (tests marked ``not gpu``):
                   the one of the state before rounding, and by its drift over
                   many tokens exceeding one rounding of the exact state.
 
+* ``branch``      branch/fork (rows continue from other rows' states) and
+                  restore-to-position [guide §"The State-Storage Bottleneck in
+                  Branching Workloads", §"What a Replay-First Design
+                  Implies"].  Pinned by recomputing every row's state from its
+                  own token lineage (a list of tokens copied at each branch),
+                  and by the identity / single-parent / full-window special
+                  cases.
+
 No function here is "parity unpinned".
 """
-from . import bookkeeping, codecs, gdn, mamba2, quantized_state, replay, speculative  # noqa: F401
+from . import bookkeeping, branch, codecs, gdn, mamba2, quantized_state, replay, speculative  # noqa: F401

@@ -22,6 +22,10 @@ implements, written per sequence in plain integers:
 * rollback (n_reject): refused (STATE) unless 0 <= n_reject <= pending; else
   len += pending - n_reject and pending = 0.  Nothing else moves.
 * flush: refused (STATE) while drafts are pending; folds a non-empty window.
+* branch (parent): row b takes row parent[b]'s pointers from before the call
+  (refused, STATE, if the parent is out of range or has pending drafts).
+* restore (keep): len = keep, for 0 <= keep <= len with no pending drafts
+  (else refused, STATE); the dropped entries are simply overwritten later.
 
 With capacity >= L + max(k, 1) the slots a call writes never overlap the slots
 a fold in the same call reads, and len + pending never exceeds L.
@@ -116,6 +120,36 @@ class WindowBook:
             if folded:
                 self._fold(b)
             out.append((OK, folded))
+        return out
+
+    def branch(self, parent):
+        """Row b takes the pointers of row parent[b] as they were before the call
+        [guide §"The State-Storage Bottleneck in Branching Workloads"].  Refused
+        (STATE) if the parent is out of range or has pending drafts."""
+        old = self.snapshot()
+        out = []
+        for b in range(self.batch):
+            p = int(parent[b])
+            if not 0 <= p < self.batch or old[2][p]:
+                out.append(ERR_STATE)
+                continue
+            self.start[b], self.len[b] = old[0][p], old[1][p]
+            self.pending[b], self.flushes[b] = old[2][p], old[3][p]
+            out.append(OK)
+        return out
+
+    def restore(self, keep):
+        """Keep only the first keep[b] committed entries of row b's window
+        [guide §"What a Replay-First Design Implies": restore to position p].
+        Refused (STATE) unless 0 <= keep <= len and no drafts are pending."""
+        out = []
+        for b in range(self.batch):
+            k = int(keep[b])
+            if self.pending[b] or not 0 <= k <= self.len[b]:
+                out.append(ERR_STATE)
+                continue
+            self.len[b] = k
+            out.append(OK)
         return out
 
     def snapshot(self):

@@ -179,3 +179,13 @@ def accept_counts(batch: int, rnd: int, k: int, seed: int = 0) -> torch.Tensor:
     """Accepted draft-prefix length per sequence, uniform on {0, ..., k}, int32."""
     return torch.randint(0, k + 1, (batch,), generator=_generator(seed, "accept", int(rnd), int(k)),
                          dtype=torch.int32)
+
+
+# ------------------------------------------------------------------ branching
+def branch_parents(batch: int, step: int, seed: int = 0, keep: float = 0.5) -> torch.Tensor:
+    """A beam-search-like parent map, int32 [batch]: each row keeps its own history
+    with probability ``keep``, else continues from a uniformly drawn row."""
+    g = _generator(seed, "branch", int(step))
+    own = torch.rand(batch, generator=g, dtype=torch.float64) < keep
+    other = torch.randint(0, batch, (batch,), generator=g, dtype=torch.int64)
+    return torch.where(own, torch.arange(batch), other).to(torch.int32)
