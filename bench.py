@@ -503,6 +503,76 @@ def speculative_leg(work, rounds=48, warmup=4, k=4):
             "speedup_vs_snapshot": round(el_base / el, 3)}
 
 
+def branch_leg(work, steps=48, warmup=8, keep=0.5):
+    """Beam-search-like decode: before every token each sequence continues from a
+    seeded parent (itself with probability `keep`, else a uniformly drawn
+    sequence), then one decode step.  Replay: rssm_branch on a branching layer
+    (windows copied, checkpoint slots shared) + decode.  Baseline: the
+    conventional design, which must give every re-parented sequence its own copy
+    of the parent's full state (a gather of those rows) before its step."""
+    import copy
+    from hybrid_ssm_decode_replayssm_b200 import rssm
+    B = work.shape.batch
+    ar = torch.arange(B, device=work.dev)
+    parents = [si.branch_parents(B, t, work.seed, keep).to(work.dev) for t in range(16)]
+    moved = [torch.nonzero(p != ar).flatten() for p in parents]
+    srcs = [p.long()[m] for p, m in zip(parents, moved)]
+    desc = copy.copy(work.desc)
+    desc.branching = 1
+    ck = torch.zeros((2 * B,) + tuple(work.h0.shape[1:]), dtype=torch.float32, device=work.dev)
+    ck[:B] = work.h0
+    layer = (rssm.ReplayLayer(desc, ck, work.A, work.D) if work.name == "mamba2"
+             else rssm.ReplayLayer(desc, ck))
+    out = torch.empty(work.out_shape, device=work.dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for t in range(warmup):
+        layer.branch(parents[t % 16])
+        layer.decode_step(work.pool[t % POOL], out)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    br = [(ev(), ev()) for _ in range(steps)]
+    e0.record()
+    for t in range(steps):
+        br[t][0].record()
+        layer.branch(parents[t % 16])
+        br[t][1].record()
+        layer.decode_step(work.pool[t % POOL], out)
+    e1.record()
+    torch.cuda.synchronize()
+    el = e0.elapsed_time(e1) / 1e3
+    branch_us = statistics.mean(a.elapsed_time(b) for a, b in br) * 1e3
+    status = layer.get_status()
+    del layer, ck
+    torch.cuda.empty_cache()
+    base = work.layer()
+    state = work.h0.clone()
+
+    def conv_step(t):
+        m = moved[t % 16]
+        state.index_copy_(0, m, state.index_select(0, srcs[t % 16]))
+        base.conventional_step(state, state, work.pool[t % POOL], out)
+    for t in range(warmup):
+        conv_step(t)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for t in range(steps):
+        conv_step(t)
+    e1.record()
+    torch.cuda.synchronize()
+    el_base = e0.elapsed_time(e1) / 1e3
+    del base, state
+    torch.cuda.empty_cache()
+    frac = statistics.mean(float(m.numel()) / B for m in moved)
+    return {"steps": steps, "reparented_fraction": round(frac, 3), "tokens_per_s": round(B * steps / el, 1),
+            "step_us": round(el / steps * 1e6, 2), "branch_us": round(branch_us, 2), "status_bits": status,
+            "conventional_baseline": {"tokens_per_s": round(B * steps / el_base, 1),
+                                      "step_us": round(el_base / steps * 1e6, 2),
+                                      "how": "gather the parents' full states into the re-parented rows, "
+                                             "then a conventional step"},
+            "speedup_vs_conventional": round(el_base / el, 3)}
+
+
 def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6):
     """Replay decode tokens/s with the fp32 checkpoint read directly and with an
     FP8 / NVFP4 read copy, per window length (checkpoint and tokens of `base`)."""
@@ -619,7 +689,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
-    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state,graph",
+    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state,graph,branch",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -701,7 +771,7 @@ def main():
     if "e2e" in legs:
         del e2e_layer
     gw = None
-    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state", "graph"}:
+    if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state", "graph", "branch"}:
         gw = GDNWork(dev, seed, args.batch)
     if world == 1 and "gdn" in legs and gw is not None:
         gl = gw.layer()
@@ -725,6 +795,11 @@ def main():
         if gw is not None:
             extras["speculative"]["gdn"] = speculative_leg(gw)
             torch.cuda.empty_cache()
+    if world == 1 and "branch" in legs:
+        extras["branch"] = {"how": "beam-search-like: each sequence re-parented with probability 1/2 before "
+                                   "every token", work.name: branch_leg(work)}
+        if gw is not None:
+            extras["branch"]["gdn"] = branch_leg(gw)
     if world == 1 and "read_copy" in legs:
         extras["read_copy"] = {work.name: read_copy_leg(work)}
         if gw is not None:

@@ -111,36 +111,6 @@ __host__ __device__ inline Layout make_layout(int L, int hc) {
   return y;
 }
 
-struct RowPlan {
-  int st, n;
-  bool refuse, pre, post;
-  unsigned bit;
-};
-__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
-  RowPlan r;
-  r.st = a.start[b];
-  r.n = a.len[b];
-  const int pend = a.pending[b];
-  r.refuse = r.pre = r.post = false;
-  r.bit = 0;
-  if (a.mode == kFlush) {
-    if (a.mask != nullptr && a.mask[b] == 0) r.refuse = true;
-    else if (pend != 0) { r.refuse = true; r.bit = RSSM_STATUS_STATE; }
-    else if (r.n == 0) r.refuse = true;
-    else r.pre = true;
-  } else if (pend != 0) {
-    r.refuse = true;
-    r.bit = RSSM_STATUS_STATE;
-  } else {
-    r.pre = r.n + a.m > a.L;
-    if (r.pre && !a.auto_flush) {
-      r.refuse = true;
-      r.bit = RSSM_STATUS_CAPACITY;
-    }
-    r.post = !r.refuse && a.mode == kDecode && a.auto_flush && ((r.pre ? 0 : r.n) + 1 == a.L);
-  }
-  return r;
-}
 
 // Quantise two state rows held in the 8-lane row mapping (lane j of the row's
 // lane group holds columns 32 c + 4 j .. + 3, c = 0..3) into the read copy,
@@ -287,7 +257,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       } else {
         const int jh = unit >> 1, hf = unit & 1;
         const int h = chunk * hc + jh;
-        const size_t bh = (size_t)b * a.H + h;
+        const size_t bh = (size_t)b * a.H + h, sbh = (size_t)rp.src * a.H + h;
         const bool fold = rp.pre || rp.post;
         // cached w rows: the reads of the committed entries, and the folds of
         // layers that fold with them
@@ -297,10 +267,10 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         uint8_t *dst = smem + s * Y.stage_bytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + nw * HALF * 4 + (nv + mv) * VHROW));
         if constexpr (RF == RSSM_READ_FP32) {
-          bulk_g2s(dst, a.hc + (bh * DV + hf * HALF) * DK, TB, &full[s]);
+          bulk_g2s(dst, a.hc + (sbh * DV + hf * HALF) * DK, TB, &full[s]);
         } else {
-          bulk_g2s(dst, a.rc_codes + (bh * DV + hf * HALF) * RB, TB, &full[s]);
-          bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + (bh * DV + hf * HALF) * SR, SB, &full[s]);
+          bulk_g2s(dst, a.rc_codes + (sbh * DV + hf * HALF) * RB, TB, &full[s]);
+          bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + (sbh * DV + hf * HALF) * SR, SB, &full[s]);
         }
         const int c1 = rp.n < cap - rp.st ? rp.n : cap - rp.st;   // ring segment lengths
         if (nw > 0) {
@@ -528,7 +498,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           else failed = true;
           continue;
         }
-        const size_t row_base = bh * DV + hf * HALF;   // first state row of this unit
+        // first state row of this unit in the checkpoint slot read (src) and in
+        // the one a fold writes (dst)
+        const size_t src_base = ((size_t)rp.src * a.H + h) * DV + hf * HALF;
+        const size_t row_base = ((size_t)rp.dst * a.H + h) * DV + hf * HALF;
+        const float *hc_src = a.hc + src_base * DK;
         float *hc_rows = a.hc + row_base * DK;
         uint8_t *rc = kResolve ? a.rc_codes + row_base * RB : nullptr;
         float4 f[2][4];   // fp32 state rows (fp32 layers: the tile; re-solving layers: fold units)
@@ -538,7 +512,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             for (int r = 0; r < 2; ++r)
 #pragma unroll
               for (int c = 0; c < 4; ++c)
-                f[r][c] = ld_stream(hc_rows + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8);
+                f[r][c] = ld_stream(hc_src + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8);
           }
         }
         // fold scalars are single-buffered: all warps must be done with the previous head's

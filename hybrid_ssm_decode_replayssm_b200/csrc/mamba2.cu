@@ -154,39 +154,6 @@ __device__ __forceinline__ void outputs(const float4 (&v)[Tile<P, N, W>::NLD], c
   }
 }
 
-// Row decision shared by the producer and the consumers of a replay CTA (both
-// read the same pointers, so they take the same branch).
-struct RowPlan {
-  int st, n;
-  bool refuse, pre, post;
-  unsigned bit;
-};
-__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
-  RowPlan r;
-  r.st = a.start[b];
-  r.n = a.len[b];
-  const int pend = a.pending[b];
-  r.refuse = r.pre = r.post = false;
-  r.bit = 0;
-  if (a.mode == kFlush) {
-    if (a.mask != nullptr && a.mask[b] == 0) r.refuse = true;
-    else if (pend != 0) { r.refuse = true; r.bit = RSSM_STATUS_STATE; }
-    else if (r.n == 0) r.refuse = true;
-    else r.pre = true;
-  } else if (pend != 0) {
-    r.refuse = true;
-    r.bit = RSSM_STATUS_STATE;
-  } else {
-    r.pre = r.n + a.m > a.L;
-    if (r.pre && !a.auto_flush) {
-      r.refuse = true;
-      r.bit = RSSM_STATUS_CAPACITY;
-    }
-    r.post = !r.refuse && a.mode == kDecode && a.auto_flush && ((r.pre ? 0 : r.n) + 1 == a.L);
-  }
-  return r;
-}
-
 // Decode heads of read-copy layers (bf16 inputs, headdim 64, dstate 128) take
 // the tensor-core path: y = h C as mma.sync m16n8k16 (f16 x f16 -> fp32), one
 // warp per 16-row tile, four warps per head.  The dequantised codes are exact
@@ -356,14 +323,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         mbar_arrive(&full[s]);
       } else {
         const int h = g * a.hpg + chunk * hc + jh;
-        const size_t bh = (size_t)b * a.H + h;
+        const size_t bh = (size_t)b * a.H + h, sbh = (size_t)rp.src * a.H + h;
         uint8_t *dst = smem + s * stage_bytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(TB + SB + (m + rp.n) * XROW));
         if constexpr (RF == RSSM_READ_FP32) {
-          bulk_g2s(dst, a.hc + bh * P * N, TB, &full[s]);
+          bulk_g2s(dst, a.hc + sbh * P * N, TB, &full[s]);
         } else {
-          bulk_g2s(dst, a.rc_codes + bh * TB, TB, &full[s]);
-          bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + bh * SB, SB, &full[s]);
+          bulk_g2s(dst, a.rc_codes + sbh * TB, TB, &full[s]);
+          bulk_g2s(dst + TB, reinterpret_cast<const uint8_t *>(a.rc_scales) + sbh * SB, SB, &full[s]);
         }
         if (rp.n > 0) {
           const Tin *src = xring + bh * cap * P;
@@ -554,9 +521,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       if (rp.refuse) {
         if (!wait_stage()) break;
       } else {
-        const size_t bh = bh0 + jh;
-        float *hc_tile = a.hc + bh * P * N;
-        uint8_t *rc = (RF != RSSM_READ_FP32) ? a.rc_codes + bh * TB : nullptr;
+        // checkpoint slots: read (src) and written by a fold (dst)
+        const size_t sbh = (size_t)rp.src * a.H + h, dbh = (size_t)rp.dst * a.H + h;
+        const float *hc_src = a.hc + sbh * P * N;
+        float *hc_dst = a.hc + dbh * P * N;
+        uint8_t *rc = (RF != RSSM_READ_FP32) ? a.rc_codes + dbh * TB : nullptr;
         const float *hs = ssc + jh * HS;
         const float *hcoef = hs, *hdec = hs + MAXM * 32, *hfw = hs + MAXM * 32 + MAXM;
         const float *hdecf = hfw + 64;
@@ -639,7 +608,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             if constexpr (RF != RSSM_READ_FP32) {
               if (pre || post) {
 #pragma unroll
-                for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_tile + (size_t)(row0 + l * T::RPI) * N + c0);
+                for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_src + (size_t)(row0 + l * T::RPI) * N + c0);
               }
             }
             float4 v[T::NLD];
@@ -653,11 +622,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 #pragma unroll
               for (int l = 0; l < T::NLD; ++l) {
                 const int row = row0 + l * T::RPI;
-                if (!post) st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+                if (!post) st_stream(hc_dst + (size_t)row * N + c0, f[l]);
                 if constexpr (RF == RSSM_READ_FP32)
                   v[l] = f[l];
                 else
-                  v[l] = quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+                  v[l] = quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, dbh * P + row, N, c0, lane);
               }
             } else {
 #pragma unroll
@@ -686,9 +655,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
 #pragma unroll
               for (int l = 0; l < T::NLD; ++l) {
                 const int row = row0 + l * T::RPI;
-                st_stream(hc_tile + (size_t)row * N + c0, f[l]);
+                st_stream(hc_dst + (size_t)row * N + c0, f[l]);
                 if constexpr (RF != RSSM_READ_FP32)
-                  quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, bh * P + row, N, c0, lane);
+                  quantize4<RF, T::LPR>(f[l], rc + (size_t)row * RB, a.rc_scales, dbh * P + row, N, c0, lane);
               }
             }
           }

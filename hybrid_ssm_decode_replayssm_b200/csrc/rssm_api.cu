@@ -79,8 +79,9 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
   const size_t B = d->batch, H = d->nheads, R = d->headdim, C = d->dstate;
   const size_t cap = d->window + (d->max_draft > 1 ? d->max_draft : 1);
   const size_t esz = d->in_dtype == RSSM_BF16 ? 2 : 4;
+  const size_t nslots = d->branching ? 2 * B : B;   // checkpoint slots
   L->cap = cap;
-  *ckpt = B * H * R * C * sizeof(float);
+  *ckpt = nslots * H * R * C * sizeof(float);
   size_t off = 0;
   if (d->kind == RSSM_MAMBA2) {
     const size_t G = d->ngroups;
@@ -94,17 +95,21 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
     L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf [B,H,cap]
     L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf [B,H,2,cap,dv/2]
   }
+  if (d->branching) {   // a copy of the ring regions for rssm_branch
+    L->branch_scratch_off = off;
+    off = align256(off + off);
+  }
   *buf = off;
   if (d->read_fmt == RSSM_READ_FP32) {
     *rc = 0;
   } else if (d->read_fmt == RSSM_READ_FP8_E4M3_ROW) {
     L->rc_codes_off = 0;
-    L->rc_scales_off = align256(B * H * R * C);
-    *rc = align256(L->rc_scales_off + B * H * R * sizeof(float));
+    L->rc_scales_off = align256(nslots * H * R * C);
+    *rc = align256(L->rc_scales_off + nslots * H * R * sizeof(float));
   } else {
     L->rc_codes_off = 0;
-    L->rc_scales_off = align256(B * H * R * C / 2);
-    *rc = align256(L->rc_scales_off + B * H * R * (C / 16));
+    L->rc_scales_off = align256(nslots * H * R * C / 2);
+    *rc = align256(L->rc_scales_off + nslots * H * R * (C / 16));
   }
   off = 0;
   L->meta_start_off = off; off = align256(off + B * 4);
@@ -113,6 +118,12 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
   L->meta_flushes_off = off; off = align256(off + B * 4);
   L->meta_arrivals_off = off; off = align256(off + B * 4);
   L->meta_status_off = off; off = align256(off + 4);
+  if (d->branching) {
+    L->meta_slot_off = off; off = align256(off + B * 4);
+    L->meta_dst_off = off; off = align256(off + B * 4);
+    L->meta_seen_off = off; off = align256(off + B * 4);
+    L->meta_work_off = off; off = align256(off + 5 * B * 4);
+  }
   *meta = off;
 }
 
@@ -129,6 +140,10 @@ rssm::StepArgs step_args(const rssm_handle *h, int mode, int m) {
   a.out_scale = d.out_scale;
   a.A = h->A; a.D = h->D;
   a.hc = h->ckpt;
+  if (d.branching) {
+    a.slot = reinterpret_cast<const int32_t *>(h->meta + h->lay.meta_slot_off);
+    a.dst = reinterpret_cast<const int32_t *>(h->meta + h->lay.meta_dst_off);
+  }
   a.rc_codes = h->rc ? h->rc + h->lay.rc_codes_off : nullptr;
   a.rc_scales = h->rc ? h->rc + h->lay.rc_scales_off : nullptr;
   a.buf0 = h->buf + h->lay.buf_off[0];
@@ -162,6 +177,19 @@ int check_inputs(const rssm_handle *h, const void *const *in, const void *out) {
   return RSSM_OK;
 }
 
+int32_t *meta_i32(const rssm_handle *h, size_t off) { return reinterpret_cast<int32_t *>(h->meta + off); }
+
+// Layers that branch: before each replay launch, give the rows that fold in it
+// a free checkpoint slot (no-op otherwise).
+int plan_slots_for(rssm_handle *h, const rssm::StepArgs &a, cudaStream_t s) {
+  if (!h->d.branching) return RSSM_OK;
+  cudaError_t e = rssm::plan_slots(a, meta_i32(h, h->lay.meta_slot_off), meta_i32(h, h->lay.meta_dst_off),
+                                   meta_i32(h, h->lay.meta_seen_off), meta_i32(h, h->lay.meta_work_off), s);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "slot planner launch");
+  return RSSM_OK;
+}
+
 int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *out,
                 const int32_t *mask, cudaStream_t s) {
   rssm::StepArgs a = step_args(h, mode, m);
@@ -169,6 +197,8 @@ int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *ou
     for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
   a.out = static_cast<float *>(out);
   a.mask = mask;
+  int rc = plan_slots_for(h, a, s);
+  if (rc) return rc;
   cudaError_t e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, s)
                                            : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, s);
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -227,6 +257,12 @@ int rssm_reset(rssm_handle *h, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   cudaError_t e = cudaMemsetAsync(h->meta, 0, h->meta_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(meta)");
+  if (h->d.branching) {
+    e = rssm::init_slots(h->d.batch, meta_i32(h, h->lay.meta_slot_off), meta_i32(h, h->lay.meta_dst_off),
+                         (cudaStream_t)stream);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return cuda_fail(e, "slot init launch");
+  }
   return ok();
 }
 
@@ -277,7 +313,7 @@ int rssm_quantize_read_copy(rssm_handle *h, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!h->rc) return fail(RSSM_ERR_STATE, "handle has no read copy (read_fmt = RSSM_READ_FP32)");
   rssm::QuantArgs q;
-  q.rows = (size_t)h->d.batch * h->d.nheads * h->d.headdim;
+  q.rows = (size_t)h->d.batch * (h->d.branching ? 2 : 1) * h->d.nheads * h->d.headdim;
   q.C = h->d.dstate;
   q.hc = h->ckpt;
   q.codes = h->rc + h->lay.rc_codes_off;
@@ -348,6 +384,71 @@ int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev, c
                       : rssm::gdn_conventional(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "quantized-state conventional kernel launch");
+  return ok();
+}
+
+int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!parent_dev) return fail(RSSM_ERR_INVALID_ARG, "parent is NULL");
+  if (!h->d.branching) return fail(RSSM_ERR_STATE, "handle was created with branching = 0");
+  rssm::BranchArgs b;
+  std::memset(&b, 0, sizeof b);
+  const rssm_layer_desc &d = h->d;
+  b.B = d.batch;
+  b.slot = meta_i32(h, h->lay.meta_slot_off);
+  b.dst = meta_i32(h, h->lay.meta_dst_off);
+  b.seen = meta_i32(h, h->lay.meta_seen_off);
+  int32_t *work = meta_i32(h, h->lay.meta_work_off);
+  b.freelist = work;
+  b.eff = work + 4 * (size_t)d.batch;
+  b.start = meta_i32(h, h->lay.meta_start_off);
+  b.len = meta_i32(h, h->lay.meta_len_off);
+  b.pending = meta_i32(h, h->lay.meta_pending_off);
+  b.flushes = meta_i32(h, h->lay.meta_flushes_off);
+  b.status = reinterpret_cast<uint32_t *>(h->meta + h->lay.meta_status_off);
+  // each ring region is [B][outer][cap][entry]
+  const int H = d.nheads;
+  const int esz = d.in_dtype == RSSM_BF16 ? 2 : 4;
+  if (d.kind == RSSM_MAMBA2) {
+    const int outer[3] = {H, d.ngroups, H}, entry[3] = {d.headdim * esz, d.dstate * esz, 4};
+    b.nreg = 3;
+    for (int r = 0; r < 3; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
+  } else {   // k [H][cap][dk] | v [2H][cap][dv/2] | g, beta [H][cap] | w [2H][cap][dv/2] fp32
+    const int outer[5] = {H, 2 * H, H, H, 2 * H};
+    const int entry[5] = {d.dstate * esz, d.headdim / 2 * esz, 4, 4, d.headdim / 2 * 4};
+    b.nreg = 5;
+    for (int r = 0; r < 5; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
+  }
+  b.cap = (int)h->lay.cap;
+  for (int r = 0; r < b.nreg; ++r) {
+    b.ring[r] = h->buf + h->lay.buf_off[r];
+    b.scratch[r] = h->buf + h->lay.branch_scratch_off + h->lay.buf_off[r];
+  }
+  cudaError_t e = rssm::branch_rows(b, parent_dev, work, (cudaStream_t)stream);
+  g_launches.fetch_add(3, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "branch launches");
+  return ok();
+}
+
+int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!keep_dev) return fail(RSSM_ERR_INVALID_ARG, "keep is NULL");
+  rssm::StepArgs a = step_args(h, rssm::kDecode, 0);
+  cudaError_t e = rssm::restore_rows(a.B, keep_dev, a.len, a.pending, a.status, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "restore launch");
+  return ok();
+}
+
+int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!out_dev) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
+  if (!h->d.branching) return fail(RSSM_ERR_STATE, "handle was created with branching = 0");
+  cudaError_t e = rssm::effective_slots(h->d.batch, meta_i32(h, h->lay.meta_slot_off),
+                                        meta_i32(h, h->lay.meta_dst_off), meta_i32(h, h->lay.meta_seen_off),
+                                        meta_i32(h, h->lay.meta_flushes_off), out_dev, (cudaStream_t)stream);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "slot lookup launch");
   return ok();
 }
 
@@ -439,6 +540,8 @@ extern "C" int rssm_decode_step_static_scratch(rssm_handle *h, const void *const
   for (int i = 0; i < n_inputs(h); ++i) a.in[i] = in[i];
   a.out = static_cast<float *>(out_dev);
   a.arrivals = arrivals;
+  rc = plan_slots_for(h, a, (cudaStream_t)stream);
+  if (rc) return rc;
   e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream)
                                : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -13,6 +13,45 @@ namespace rssm {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// ------------------------------------------------------------ row plan
+// What one call does to sequence b, decided from its pointers alone (the
+// window rules of rssm.h): refuse the row (with a status bit), fold the
+// committed window before appending (pre), fold the full window after the
+// decode (post).  src / dst: the checkpoint slot the row reads, and the one a
+// fold of this call writes (both b unless the layer branches).
+struct RowPlan {
+  int st, n, src, dst;
+  bool refuse, pre, post;
+  unsigned bit;
+};
+__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
+  RowPlan r;
+  r.st = a.start[b];
+  r.n = a.len[b];
+  r.src = a.slot ? a.slot[b] : b;
+  r.dst = a.dst ? a.dst[b] : b;
+  const int pend = a.pending[b];
+  r.refuse = r.pre = r.post = false;
+  r.bit = 0;
+  if (a.mode == kFlush) {
+    if (a.mask != nullptr && a.mask[b] == 0) r.refuse = true;
+    else if (pend != 0) { r.refuse = true; r.bit = RSSM_STATUS_STATE; }
+    else if (r.n == 0) r.refuse = true;
+    else r.pre = true;
+  } else if (pend != 0) {
+    r.refuse = true;
+    r.bit = RSSM_STATUS_STATE;
+  } else {
+    r.pre = r.n + a.m > a.L;
+    if (r.pre && !a.auto_flush) {
+      r.refuse = true;
+      r.bit = RSSM_STATUS_CAPACITY;
+    }
+    r.post = !r.refuse && a.mode == kDecode && a.auto_flush && ((r.pre ? 0 : r.n) + 1 == a.L);
+  }
+  return r;
+}
+
 // ---------------------------------------------------------------- loads
 // The checkpoint is streamed once per call: keep it out of L1 and mark it
 // evict-first in L2 so the window buffers (re-read every step) stay cached.

@@ -27,8 +27,10 @@ struct StepArgs {
   float out_scale;       // GDN
   // parameters (Mamba-2)
   const float *A, *D;
-  // checkpoint and read copy
+  // checkpoint and read copy (with branching: 2B slots; row b reads slot[b]
+  // and a fold of row b writes slot dst[b]; without: both NULL, slot b = row b)
   float *hc;
+  const int32_t *slot, *dst;
   uint8_t *rc_codes;
   void *rc_scales;
   // ring buffers (layer specific, see rssm.h)
@@ -78,6 +80,35 @@ cudaError_t rollback(int B, const int32_t *n_reject, int32_t *len, int32_t *pend
 cudaError_t gather_bookkeeping(int B, const int32_t *start, const int32_t *len,
                                const int32_t *pending, const int32_t *flushes, int32_t *out,
                                cudaStream_t s);
+
+// Branching (rows sharing checkpoint slots).  BranchArgs describes the meta
+// arrays and the ring regions copied when a row takes another row's window.
+struct BranchArgs {
+  int B;
+  int32_t *slot, *dst, *seen, *freelist, *eff;   // [B] [B] [B] [2B] [B]
+  int32_t *start, *len, *pending, *flushes;
+  uint32_t *status;
+  int nreg;                   // ring regions in buf
+  int cap;                    // ring capacity (entries)
+  uint8_t *ring[5];           // region bases
+  uint8_t *scratch[5];        // their copies in the branch scratch
+  // A region is [B][outer][cap][entry bytes]: one sequence's row holds `outer`
+  // rings (heads, groups or head halves) of cap entries each.
+  int outer[5];
+  int entry_bytes[5];
+};
+// Before a replay launch: adopt the slots written by the previous launch's
+// folds, then give every row that folds in this launch a free slot.
+cudaError_t plan_slots(const StepArgs &a, int32_t *slot, int32_t *dst, int32_t *seen, int32_t *freelist,
+                       cudaStream_t s);
+// rssm_branch: bookkeeping gather, then the window copy through the scratch.
+// tmp: int32 [4B] scratch.
+cudaError_t branch_rows(const BranchArgs &b, const int32_t *parent, int32_t *tmp, cudaStream_t s);
+cudaError_t restore_rows(int B, const int32_t *keep, int32_t *len, const int32_t *pending,
+                         uint32_t *status, cudaStream_t s);
+cudaError_t init_slots(int B, int32_t *slot, int32_t *dst, cudaStream_t s);
+cudaError_t effective_slots(int B, const int32_t *slot, const int32_t *dst, const int32_t *seen,
+                            const int32_t *flushes, int32_t *out, cudaStream_t s);
 
 bool mamba2_supported(int R, int C);
 bool gdn_supported(int R, int C);

@@ -33,6 +33,7 @@ EXPORTED = [
     "rssm_quantize_read_copy", "rssm_conventional_step", "rssm_get_bookkeeping",
     "rssm_get_status", "rssm_last_error_string", "rssm_launch_count",
     "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
+    "rssm_branch", "rssm_restore", "rssm_get_slots",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -41,7 +42,7 @@ class LayerDesc(C.Structure):
     _fields_ = [("kind", C.c_int), ("batch", C.c_int), ("nheads", C.c_int), ("ngroups", C.c_int),
                 ("headdim", C.c_int), ("dstate", C.c_int), ("window", C.c_int),
                 ("max_draft", C.c_int), ("in_dtype", C.c_int), ("read_fmt", C.c_int),
-                ("auto_flush", C.c_int), ("out_scale", C.c_float)]
+                ("auto_flush", C.c_int), ("out_scale", C.c_float), ("branching", C.c_int)]
 
 
 class Layout(C.Structure):
@@ -49,7 +50,9 @@ class Layout(C.Structure):
                 ("rc_scales_off", C.c_size_t), ("meta_start_off", C.c_size_t),
                 ("meta_len_off", C.c_size_t), ("meta_pending_off", C.c_size_t),
                 ("meta_flushes_off", C.c_size_t), ("meta_arrivals_off", C.c_size_t),
-                ("meta_status_off", C.c_size_t)]
+                ("meta_status_off", C.c_size_t), ("meta_slot_off", C.c_size_t),
+                ("meta_dst_off", C.c_size_t), ("meta_seen_off", C.c_size_t),
+                ("meta_work_off", C.c_size_t), ("branch_scratch_off", C.c_size_t)]
 
 
 _LIB = None
@@ -79,6 +82,9 @@ def lib():
         L.rssm_conventional_step.argtypes = [vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_conventional_step_quantized.argtypes = [vp, vp, vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_get_bookkeeping.argtypes = [vp, vp, vp]
+        L.rssm_branch.argtypes = [vp, vp, vp]
+        L.rssm_restore.argtypes = [vp, vp, vp]
+        L.rssm_get_slots.argtypes = [vp, vp, vp]
         L.rssm_get_status.argtypes = [vp, C.POINTER(C.c_uint32), i32, vp]
         for name in EXPORTED:
             getattr(L, name).restype = C.c_int
@@ -118,9 +124,10 @@ def _ptr_array(tensors):
 
 
 def make_desc(kind, batch, nheads, headdim, dstate, ngroups=1, window=16, max_draft=4,
-              in_dtype=RSSM_BF16, read_fmt=RSSM_READ_FP32, auto_flush=True, out_scale=1.0):
+              in_dtype=RSSM_BF16, read_fmt=RSSM_READ_FP32, auto_flush=True, out_scale=1.0,
+              branching=False):
     return LayerDesc(kind, batch, nheads, ngroups, headdim, dstate, window, max_draft,
-                     in_dtype, read_fmt, int(bool(auto_flush)), float(out_scale))
+                     in_dtype, read_fmt, int(bool(auto_flush)), float(out_scale), int(bool(branching)))
 
 
 def workspace_size(desc: LayerDesc):
@@ -135,7 +142,9 @@ class ReplayLayer:
     """One SSM layer's ReplaySSM storage on one GPU, with torch-owned buffers.
 
     ``ckpt`` is the fp32 checkpoint tensor [B, H, R, C] on the device (kept by
-    reference: the library folds windows into it in place).
+    reference: the library folds windows into it in place).  A branching
+    layer's checkpoint has 2B slots, [2B, H, R, C]: the caller fills the first
+    B, and ``checkpoint_rows()`` gathers the one each sequence reads.
     """
 
     def __init__(self, desc: LayerDesc, ckpt: torch.Tensor, A=None, D=None, stream=None):
@@ -215,6 +224,25 @@ class ReplayLayer:
                     torch.zeros((B, H, R, Cc // 16), dtype=torch.uint8, device=dev))
         raise ValueError("layer has no low-precision format")
 
+    def branch(self, parent, stream=None):
+        """Sequence b continues from sequence parent[b] (device int32 [B])."""
+        check(lib().rssm_branch(self.handle, parent.data_ptr(), _stream(stream)))
+
+    def restore(self, keep, stream=None):
+        """Sequence b keeps the first keep[b] committed tokens of its window."""
+        check(lib().rssm_restore(self.handle, keep.data_ptr(), _stream(stream)))
+
+    def get_slots(self, stream=None) -> torch.Tensor:
+        out = torch.empty(self.desc.batch, dtype=torch.int32, device=self.ckpt.device)
+        check(lib().rssm_get_slots(self.handle, out.data_ptr(), _stream(stream)))
+        return out
+
+    def checkpoint_rows(self, stream=None) -> torch.Tensor:
+        """The checkpoint each sequence reads, [B, H, R, C] (a copy)."""
+        if not self.desc.branching:
+            return self.ckpt.clone()
+        return self.ckpt.index_select(0, self.get_slots(stream).long())
+
     def get_bookkeeping(self, stream=None) -> torch.Tensor:
         out = torch.empty((4, self.desc.batch), dtype=torch.int32, device=self.ckpt.device)
         check(lib().rssm_get_bookkeeping(self.handle, out.data_ptr(), _stream(stream)))
@@ -232,7 +260,7 @@ class ReplayLayer:
     def read_copy_views(self):
         """(codes uint8, scales) views of the read copy, shaped per rssm.h."""
         d, lay = self.desc, self.layout
-        B, H, R, Cc = d.batch, d.nheads, d.headdim, d.dstate
+        B, H, R, Cc = d.batch * (2 if d.branching else 1), d.nheads, d.headdim, d.dstate
         rc = self.read_copy
         if d.read_fmt == RSSM_READ_FP8_E4M3_ROW:
             codes = rc[: B * H * R * Cc].view(B, H, R, Cc)

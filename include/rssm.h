@@ -107,6 +107,7 @@ typedef struct {
   int read_fmt;    /* RSSM_READ_*                                             */
   int auto_flush;  /* nonzero: fold the window when it fills / must make room */
   float out_scale; /* GDN output scale (1.0 = none); ignored for Mamba-2      */
+  int branching;   /* nonzero: rows may share checkpoints (rssm_branch)       */
 } rssm_layer_desc;
 
 /*
@@ -128,6 +129,19 @@ typedef struct {
  * Ring entry i (0-based, oldest first) of sequence b lives in slot
  * (start[b] + i) % cap.  len = committed entries, pending = unverified
  * drafts after them, flushes = number of folds so far.
+ *
+ * Branching layers (desc.branching != 0) [guide "The State-Storage
+ * Bottleneck in Branching Workloads": beam search, best-of-n and tree search
+ * spawn several continuations of one prefix]: several sequences may read one
+ * checkpoint.  The checkpoint then holds 2B slots of [H,R,C] fp32 (ckpt
+ * [2B,H,R,C]; the read copy likewise 2B slots); sequence b reads slot slot[b]
+ * (int32 meta array, slot[b] = b after rssm_reset, so the caller initialises
+ * slots 0..B-1 as the sequences' checkpoints).  A fold never writes a slot
+ * that any sequence reads: before each replay launch a planner kernel gives
+ * every sequence that folds in it a free slot (2B slots, at most B of them
+ * read, so one always exists), and the sequence moves to that slot.  meta
+ * also holds int32 dst[B], seen[B] and a work area of 5B int32 (internal),
+ * and buf a scratch copy of the ring regions (branch_scratch_off).
  */
 typedef struct {
   size_t cap;
@@ -135,13 +149,17 @@ typedef struct {
   size_t rc_codes_off, rc_scales_off;
   size_t meta_start_off, meta_len_off, meta_pending_off, meta_flushes_off,
       meta_arrivals_off, meta_status_off;
+  /* branching layers only (0 otherwise) */
+  size_t meta_slot_off, meta_dst_off, meta_seen_off, meta_work_off;
+  size_t branch_scratch_off;   /* in buf: a copy of the ring regions above */
 } rssm_layout;
 
 typedef struct rssm_handle rssm_handle;
 
 /* Sizes (bytes) of the four caller-owned device buffers for a descriptor, and
  * the layout inside them (layout may be NULL).  ckpt = the fp32 checkpoint;
- * read_copy is 0 for RSSM_READ_FP32. */
+ * read_copy is 0 for RSSM_READ_FP32.  desc.branching doubles the checkpoint
+ * and read copy (2B slots) and adds the branch scratch and meta arrays. */
 int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes,
                         size_t *buf_bytes, size_t *read_copy_bytes,
                         size_t *meta_bytes, rssm_layout *layout);
@@ -155,7 +173,8 @@ int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev,
                 void *read_copy_dev, void *meta_dev, rssm_handle **out);
 int rssm_destroy(rssm_handle *h);
 
-/* Zero the meta region (empty windows, no drafts, status clear). */
+/* Zero the meta region (empty windows, no drafts, status clear); branching
+ * layers: every sequence back to slot b. */
 int rssm_reset(rssm_handle *h, rssm_stream_t stream);
 
 /* Mamba-2 per-head parameters A[H] (< 0) and D[H], fp32 device arrays kept
@@ -212,7 +231,8 @@ int rssm_flush(rssm_handle *h, const int32_t *row_mask_dev,
 
 /*
  * Rebuild the whole low-precision read copy from the fp32 checkpoint
- * [summary ¶4].  Call after creating the handle or writing the checkpoint.
+ * [summary ¶4] (all 2B slots of a branching layer).  Call after creating
+ * the handle or writing the checkpoint.
  * RSSM_ERR_STATE if the handle has no read copy.
  */
 int rssm_quantize_read_copy(rssm_handle *h, rssm_stream_t stream);
@@ -275,6 +295,36 @@ int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev,
 #define RSSM_STATIC_SCRATCH_MAX_BATCH 65536
 int rssm_decode_step_static_scratch(rssm_handle *h, const void *const *in,
                                     void *out_dev, rssm_stream_t stream);
+
+/*
+ * Branch / fork [guide "The State-Storage Bottleneck in Branching
+ * Workloads"]: every sequence b continues from the state sequence
+ * parent_dev[b] had before the call (device int32 [B]; parent[b] == b keeps
+ * b).  All sequences move at once, as a gather.  The child shares the
+ * parent's checkpoint slot (no state is copied) and takes a copy of its
+ * window (ring entries and pointers: start, len, flushes; pending is 0); its
+ * own next fold writes a slot of its own.  A sequence whose parent is out of
+ * range or has pending drafts sets RSSM_STATUS_STATE and keeps its own state.
+ * Three kernel launches: bookkeeping, then the windows copied through the
+ * scratch (so a sequence that is both parent and child is read first).
+ * RSSM_ERR_STATE if the handle was created with branching = 0.
+ */
+int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream);
+
+/*
+ * Restore to a position [guide "What a Replay-First Design Implies": the
+ * decode loop gains "restore state to position p"]: sequence b returns to its
+ * state after the first keep_dev[b] committed tokens of its current window
+ * (the tokens since its last fold): len = keep.  Only the pointer moves.
+ * keep outside [0, len] or pending drafts: RSSM_STATUS_STATE, row unchanged.
+ * Any layer (branching or not).
+ */
+int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream);
+
+/* The checkpoint slot each sequence reads, after the folds of the calls
+ * enqueued so far (device int32 [B]); its checkpoint is ckpt slot out[b].
+ * RSSM_ERR_STATE if the handle was created with branching = 0. */
+int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream);
 
 /* Copy the per-sequence pointers into out_dev (device int32 [4, B]: start,
  * len, pending, flushes). */

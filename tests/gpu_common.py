@@ -37,25 +37,37 @@ def assert_close(got, want, tol, what=""):
     return e
 
 
-def m2_layer(shape: si.Mamba2Layer, read_fmt=rssm.RSSM_READ_FP32, auto_flush=True, seed=0, max_draft=None):
+def _ckpt(h0, branching):
+    """The device checkpoint: h0 itself, or for a branching layer 2B slots whose
+    first B hold h0."""
+    if not branching:
+        return h0.to(DEV).contiguous()
+    c = torch.zeros((2 * h0.shape[0],) + tuple(h0.shape[1:]), dtype=torch.float32, device=DEV)
+    c[: h0.shape[0]] = h0.to(DEV)
+    return c
+
+
+def m2_layer(shape: si.Mamba2Layer, read_fmt=rssm.RSSM_READ_FP32, auto_flush=True, seed=0, max_draft=None,
+             branching=False):
     A, D = si.mamba2_params(shape, seed)
     h0 = si.mamba2_checkpoint(shape, seed)
     desc = rssm.make_desc(rssm.RSSM_MAMBA2, shape.batch, shape.nheads, shape.headdim, shape.dstate,
                           ngroups=shape.ngroups, window=shape.window,
                           max_draft=shape.max_draft if max_draft is None else max_draft,
                           in_dtype=rssm.RSSM_BF16 if shape.dtype == "bf16" else rssm.RSSM_F32,
-                          read_fmt=read_fmt, auto_flush=auto_flush)
-    layer = rssm.ReplayLayer(desc, h0.to(DEV).contiguous(), A.to(DEV), D.to(DEV))
+                          read_fmt=read_fmt, auto_flush=auto_flush, branching=branching)
+    layer = rssm.ReplayLayer(desc, _ckpt(h0, branching), A.to(DEV), D.to(DEV))
     return layer, A.double().numpy(), D.double().numpy(), h0
 
 
 def gdn_layer(shape: si.GDNLayer, read_fmt=rssm.RSSM_READ_FP32, auto_flush=True, seed=0, out_scale=1.0,
-              max_draft=None):
+              max_draft=None, branching=False):
     S0 = si.gdn_checkpoint(shape, seed)
     desc = rssm.make_desc(rssm.RSSM_GDN, shape.batch, shape.nheads, shape.dv, shape.dk,
                           window=shape.window,
                           max_draft=shape.max_draft if max_draft is None else max_draft,
                           in_dtype=rssm.RSSM_BF16 if shape.dtype == "bf16" else rssm.RSSM_F32,
-                          read_fmt=read_fmt, auto_flush=auto_flush, out_scale=out_scale)
-    layer = rssm.ReplayLayer(desc, S0.to(DEV).contiguous())
+                          read_fmt=read_fmt, auto_flush=auto_flush, out_scale=out_scale,
+                          branching=branching)
+    layer = rssm.ReplayLayer(desc, _ckpt(S0, branching))
     return layer, S0

@@ -155,3 +155,44 @@ def test_null_handle_everywhere():
     assert L.rssm_flush(None, None, None) == rssm.RSSM_ERR_INVALID_ARG
     assert L.rssm_decode_step(None, None, None, None) == rssm.RSSM_ERR_INVALID_ARG
     assert L.rssm_launch_count() >= 0
+
+
+def test_workspace_layout_branching():
+    """A branching layer doubles the checkpoint and read copy (2B slots) and adds the
+    branch scratch (a copy of the ring regions) and the slot arrays."""
+    for fmt in (rssm.RSSM_READ_FP32, rssm.RSSM_READ_NVFP4):
+        code, (ck, buf, rc, meta), lay = _sizes(_desc(read_fmt=fmt))
+        code2, (ck2, buf2, rc2, meta2), lay2 = _sizes(_desc(read_fmt=fmt, branching=True))
+        assert code == code2 == rssm.RSSM_OK
+        assert ck2 == 2 * ck and (rc2 >= 2 * rc - 512)
+        assert lay2.branch_scratch_off >= lay2.buf_off[2] and lay2.branch_scratch_off % 256 == 0
+        assert buf2 >= 2 * lay2.branch_scratch_off and lay.branch_scratch_off == 0
+        B = 4
+        offs = [lay2.meta_slot_off, lay2.meta_dst_off, lay2.meta_seen_off, lay2.meta_work_off]
+        assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+        assert offs[0] > lay2.meta_status_off and meta2 >= offs[3] + 5 * B * 4
+        assert lay.meta_slot_off == lay.meta_work_off == 0
+
+
+def test_branch_calls_check_arguments():
+    L = rssm.lib()
+    fake = 1 << 20
+    h = C.c_void_p()
+    assert L.rssm_branch(None, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_restore(None, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_get_slots(None, fake, None) == rssm.RSSM_ERR_INVALID_ARG
+    d = _desc()
+    assert L.rssm_create(C.byref(d), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        assert L.rssm_branch(h, fake, None) == rssm.RSSM_ERR_STATE       # created without branching
+        assert L.rssm_get_slots(h, fake, None) == rssm.RSSM_ERR_STATE
+        assert L.rssm_restore(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+    finally:
+        L.rssm_destroy(h)
+    d = _desc(branching=True)
+    assert L.rssm_create(C.byref(d), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        assert L.rssm_branch(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+        assert L.rssm_get_slots(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
+    finally:
+        L.rssm_destroy(h)
