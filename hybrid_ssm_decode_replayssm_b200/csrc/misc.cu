@@ -129,85 +129,108 @@ __global__ void __launch_bounds__(1024) plan_slots_kernel(const StepArgs a, int3
   }
 }
 
-// rssm_branch, step 1 (one CTA): adopt pending folds; decide each row's
-// effective parent (eff = parent, or -1 when refused); gather the parents'
-// slot and pointers (all read before any is written).
-__global__ void __launch_bounds__(1024) branch_book_kernel(const BranchArgs a, const int32_t *parent,
-                                                           int32_t *tmp) {
-  const int B = a.B, nt = blockDim.x;
-  adopt_folds(B, a.slot, a.dst, a.seen, a.flushes);
-  __syncthreads();
-  for (int b = threadIdx.x; b < B; b += nt) {
-    const int p = parent[b];
-    const bool ok = p >= 0 && p < B && a.pending[p] == 0;
+// rssm_branch, two launches of one 1024-thread block per sequence.
+//
+// Pass 1 (gather): block b decides its sequence's effective parent (eff =
+// parent, or -1 when refused), gathers the parent's checkpoint slot (taking a
+// fold of the previous launch into account) and pointers into tmp [4][B], and
+// copies the live window entries of the parent's rings into b's scratch rows.
+// Nothing that pass reads is written in it.
+// Pass 2 (scatter): block b writes the gathered pointers (or, for a sequence
+// that keeps its own state, adopts its last fold's slot) and copies its
+// scratch rows into its rings.  A sequence that is both parent and child is
+// read in pass 1 before pass 2 overwrites it.
+//
+// A ring region is [B][outer][cap][entry]; the live entries of each ring are
+// (start + e) % cap, e < len.  A block walks all live words of its sequence
+// (16-byte words where the entry size allows, else 4-byte words) with flat
+// indices, four independent loads in flight per thread before their stores.
+template <typename W>
+__device__ __forceinline__ void copy_live_words(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                                int outer, int cap, int ew, int n, int st) {
+  const W *s = reinterpret_cast<const W *>(src);
+  W *d = reinterpret_cast<W *>(dst);
+  const int per_ring = n * ew;
+  const int total = outer * per_ring;
+  auto word = [&](int w) -> size_t {   // flat live-word index -> word offset in the row
+    const int o = w / per_ring, rem = w - o * per_ring;
+    const int e = rem / ew, c = rem - e * ew;
+    int idx = st + e;
+    if (idx >= cap) idx -= cap;
+    return ((size_t)o * cap + idx) * ew + c;
+  };
+  const int bd = blockDim.x;
+  for (int w0 = threadIdx.x; w0 < total; w0 += 4 * bd) {
+    size_t off[4];
+    W v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (w0 + q * bd < total) {
+        off[q] = word(w0 + q * bd);
+        v[q] = s[off[q]];
+      }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (w0 + q * bd < total) d[off[q]] = v[q];
+  }
+}
+
+__device__ __forceinline__ void copy_row(const BranchArgs &a, const uint8_t *const *src_base, size_t src_row,
+                                         uint8_t *const *dst_base, size_t dst_row, int n, int st) {
+  for (int r = 0; r < a.nreg; ++r) {
+    const int eb = a.entry_bytes[r];
+    const size_t rb = (size_t)a.outer[r] * a.cap * eb;   // one sequence's row in region r
+    const uint8_t *src = src_base[r] + src_row * rb;
+    uint8_t *dst = dst_base[r] + dst_row * rb;
+    if (eb % 16 == 0) copy_live_words<uint4>(src, dst, a.outer[r], a.cap, eb / 16, n, st);
+    else copy_live_words<uint32_t>(src, dst, a.outer[r], a.cap, eb / 4, n, st);
+  }
+}
+
+__global__ void __launch_bounds__(1024) branch_gather_kernel(const BranchArgs a, const int32_t *parent,
+                                                             int32_t *tmp) {
+  const int B = a.B, b = blockIdx.x;
+  const int p = parent[b];
+  const bool ok = p >= 0 && p < B && a.pending[p] == 0;
+  if (threadIdx.x == 0) {
     a.eff[b] = ok ? p : -1;
     if (!ok) atomicOr(a.status, (unsigned)RSSM_STATUS_STATE);
     if (ok && p != b) {
-      tmp[b] = a.slot[p];
+      const int f = a.flushes[p];
+      tmp[b] = f != a.seen[p] ? a.dst[p] : a.slot[p];
       tmp[B + b] = a.start[p];
       tmp[2 * B + b] = a.len[p];
-      tmp[3 * B + b] = a.flushes[p];
+      tmp[3 * B + b] = f;
     }
   }
-  __syncthreads();
-  for (int b = threadIdx.x; b < B; b += nt) {
-    const int p = a.eff[b];
-    if (p >= 0 && p != b) {
+  if (!ok || p == b) return;
+  const int n = a.len[p];
+  if (n > 0) copy_row(a, a.ring, (size_t)p, a.scratch, (size_t)b, n, a.start[p]);
+}
+
+__global__ void __launch_bounds__(1024) branch_scatter_kernel(const BranchArgs a, const int32_t *tmp) {
+  const int B = a.B, b = blockIdx.x;
+  const int p = a.eff[b];
+  const bool moved = p >= 0 && p != b;
+  if (threadIdx.x == 0) {
+    if (moved) {
       a.slot[b] = tmp[b];
       a.start[b] = tmp[B + b];
       a.len[b] = tmp[2 * B + b];
       a.flushes[b] = tmp[3 * B + b];
       a.seen[b] = tmp[3 * B + b];
       a.pending[b] = 0;
-    }
-  }
-}
-
-// rssm_branch, steps 2 and 3: the live window entries of every row with a
-// new parent go ring -> scratch (from the parent's rings) and then scratch ->
-// ring (into the row's), so a row that is both a parent and a child is read
-// before it is overwritten.  After step 1 the child's start and len are the
-// parent's, so both passes copy entries (start + e) % cap, e < len, of each of
-// the row's rings.  One warp per (row, ring); 16-byte words where the entry
-// size allows, else 4-byte words.
-template <bool kToScratch>
-__global__ void __launch_bounds__(256) branch_copy_kernel(const BranchArgs a) {
-  const int lane = threadIdx.x & 31;
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  int per_row = 0;
-  for (int r = 0; r < a.nreg; ++r) per_row += a.outer[r];
-  const long long total = (long long)a.B * per_row;
-  for (long long it = warp; it < total; it += nwarps) {
-    const int b = (int)(it / per_row);
-    int k = (int)(it - (long long)b * per_row);
-    const int p = a.eff[b];
-    const int n = a.len[b];
-    if (p < 0 || p == b || n == 0) continue;
-    int r = 0;
-    while (k >= a.outer[r]) k -= a.outer[r++];
-    const size_t eb = (size_t)a.entry_bytes[r];
-    const size_t rb = (size_t)a.outer[r] * a.cap * eb;   // bytes of one row in region r
-    const uint8_t *src = kToScratch ? a.ring[r] + (size_t)p * rb : a.scratch[r] + (size_t)b * rb;
-    uint8_t *dst = kToScratch ? a.scratch[r] + (size_t)b * rb : a.ring[r] + (size_t)b * rb;
-    const size_t ring0 = (size_t)k * a.cap * eb;          // this ring inside the row
-    const int st = a.start[b];
-    const int n1 = n < a.cap - st ? n : a.cap - st;       // entries before the wrap
-    for (int seg = 0; seg < 2; ++seg) {
-      const int e0 = seg ? 0 : st, cnt = seg ? n - n1 : n1;
-      if (cnt <= 0) continue;
-      const size_t off = ring0 + (size_t)e0 * eb, bytes = (size_t)cnt * eb;
-      if (eb % 16 == 0) {
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + off);
-        uint4 *d4 = reinterpret_cast<uint4 *>(dst + off);
-        for (size_t w = lane; w < bytes / 16; w += 32) d4[w] = s4[w];
-      } else {
-        const uint32_t *s1 = reinterpret_cast<const uint32_t *>(src + off);
-        uint32_t *d1 = reinterpret_cast<uint32_t *>(dst + off);
-        for (size_t w = lane; w < bytes / 4; w += 32) d1[w] = s1[w];
+    } else {
+      const int f = a.flushes[b];
+      if (f != a.seen[b]) {   // this sequence's own fold of the previous launch
+        a.slot[b] = a.dst[b];
+        a.seen[b] = f;
       }
     }
   }
+  if (!moved) return;
+  const int n = tmp[2 * B + b];
+  if (n > 0) copy_row(a, a.scratch, (size_t)b, a.ring, (size_t)b, n, tmp[B + b]);
 }
 
 __global__ void restore_kernel(int B, const int32_t *keep, int32_t *len, const int32_t *pending,
@@ -279,15 +302,10 @@ cudaError_t plan_slots(const StepArgs &a, int32_t *slot, int32_t *dst, int32_t *
 }
 
 cudaError_t branch_rows(const BranchArgs &b, const int32_t *parent, int32_t *tmp, cudaStream_t s) {
-  branch_book_kernel<<<1, 1024, 0, s>>>(b, parent, tmp);
+  branch_gather_kernel<<<dim3((unsigned)b.B), dim3(1024), 0, s>>>(b, parent, tmp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  branch_copy_kernel<true><<<dim3((unsigned)sms * 8), dim3(256), 0, s>>>(b);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  branch_copy_kernel<false><<<dim3((unsigned)sms * 8), dim3(256), 0, s>>>(b);
+  branch_scatter_kernel<<<dim3((unsigned)b.B), dim3(1024), 0, s>>>(b, tmp);
   return cudaGetLastError();
 }
 

@@ -425,7 +425,7 @@ int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream)
     b.scratch[r] = h->buf + h->lay.branch_scratch_off + h->lay.buf_off[r];
   }
   cudaError_t e = rssm::branch_rows(b, parent_dev, work, (cudaStream_t)stream);
-  g_launches.fetch_add(3, std::memory_order_relaxed);
+  g_launches.fetch_add(2, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "branch launches");
   return ok();
 }

@@ -305,15 +305,16 @@ int rssm_decode_step_static_scratch(rssm_handle *h, const void *const *in,
  * window (ring entries and pointers: start, len, flushes; pending is 0); its
  * own next fold writes a slot of its own.  A sequence whose parent is out of
  * range or has pending drafts sets RSSM_STATUS_STATE and keeps its own state.
- * Three kernel launches: bookkeeping, then the windows copied through the
- * scratch (so a sequence that is both parent and child is read first).
+ * Two kernel launches: the parents' pointers and live window entries are
+ * gathered (into the scratch), then scattered into the children, so a
+ * sequence that is both parent and child is read before it is overwritten.
  * RSSM_ERR_STATE if the handle was created with branching = 0.
  */
 int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream);
 
 /*
  * Restore to a position [guide "What a Replay-First Design Implies": the
- * decode loop gains "restore state to position p"]: sequence b returns to its
+ * decode loop can return a sequence to an earlier position]: sequence b returns to its
  * state after the first keep_dev[b] committed tokens of its current window
  * (the tokens since its last fold): len = keep.  Only the pointer moves.
  * keep outside [0, len] or pending drafts: RSSM_STATUS_STATE, row unchanged.

@@ -4,7 +4,7 @@
 best-of-n sampling and tree-structured reasoning spawn several continuations
 of one prefix, and at a branch point each continuation needs the prefix's
 state as its own.  [guide §"What a Replay-First Design Implies"]: the decode
-loop gains the primitive "restore the state to position p".
+loop can return a sequence to the state it had at an earlier position p.
 
 Readings the library implements:
 

@@ -3,8 +3,8 @@
 Beam search, best-of-n and tree search spawn several continuations of one
 prefix ("ReplaySSM: Rethinking State Storage for Faster Hybrid-Model
 Decoding", nexus-ai-blog.com guide, §"The State-Storage Bottleneck in
-Branching Workloads"), and the decode loop gains "restore the state to
-position p" (same guide, §"What a Replay-First Design Implies").  A branching
+Branching Workloads"), and the decode loop can return a sequence to the state
+it had at an earlier position (same guide, §"What a Replay-First Design Implies").  A branching
 layer lets rows share a checkpoint slot and copies only windows; folds move a
 row to a free slot.  Here random sequences of decode, branch, restore and
 flush calls run on the GPU and on the oracle (oracle.branch) side by side:
