@@ -58,6 +58,12 @@ Modules and what pins each one (tests marked ``not gpu``):
                   the one of the state before rounding, and by its drift over
                   many tokens exceeding one rounding of the exact state.
 
+* ``kda``         Kimi Delta Attention (reading: the gated delta rule with a
+                  per-key-channel gate) and its replay form.  Pinned by the
+                  gated delta rule it reduces to with equal channel gates, the
+                  explicit product of transitions (d <= 4), beta = 0 channel
+                  decay, orthonormal-key memorisation, and replay equal to the
+                  recurrence for L in {1, 2, 3, 4, 8, 16, 32}.
 * ``branch``      branch/fork (rows continue from other rows' states) and
                   restore-to-position [guide §"The State-Storage Bottleneck in
                   Branching Workloads", §"What a Replay-First Design
@@ -68,4 +74,4 @@ Modules and what pins each one (tests marked ``not gpu``):
 
 No function here is "parity unpinned".
 """
-from . import bookkeeping, branch, codecs, gdn, mamba2, quantized_state, replay, speculative  # noqa: F401
+from . import bookkeeping, branch, codecs, gdn, kda, mamba2, quantized_state, replay, speculative  # noqa: F401

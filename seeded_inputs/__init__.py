@@ -81,6 +81,21 @@ class GDNLayer:
         return replace(self, **kw)
 
 
+@dataclass(frozen=True)
+class KDALayer:
+    """Shape of one Kimi Delta Attention layer at decode time (per-channel gates)."""
+    batch: int
+    nheads: int
+    dk: int
+    dv: int
+    window: int = 16
+    dtype: str = "bf16"
+    state_std: float = 0.05
+
+    def with_(self, **kw) -> "KDALayer":
+        return replace(self, **kw)
+
+
 # Mamba-2, fp32 throughout, 64 steps from a zero checkpoint (parity workload).
 MAMBA2_TINY_F32 = Mamba2Layer(batch=4, nheads=8, headdim=64, dstate=64,
                               ngroups=1, window=16, dtype="f32", state_std=0.0)
@@ -89,6 +104,9 @@ MAMBA2_SERVING = Mamba2Layer(batch=256, nheads=128, headdim=64, dstate=128,
                              ngroups=8, window=16, dtype="bf16", state_std=0.1)
 # Gated DeltaNet decode layer at serving batch 256 (512 MiB fp32 checkpoint).
 GDN_SERVING = GDNLayer(batch=256, nheads=32, dk=128, dv=128, window=16,
+                       dtype="bf16", state_std=0.05)
+# KDA decode layer of the same shape as the GDN one.
+KDA_SERVING = KDALayer(batch=256, nheads=32, dk=128, dv=128, window=16,
                        dtype="bf16", state_std=0.05)
 
 
@@ -179,6 +197,32 @@ def accept_counts(batch: int, rnd: int, k: int, seed: int = 0) -> torch.Tensor:
     """Accepted draft-prefix length per sequence, uniform on {0, ..., k}, int32."""
     return torch.randint(0, k + 1, (batch,), generator=_generator(seed, "accept", int(rnd), int(k)),
                          dtype=torch.int32)
+
+
+# ------------------------------------------------------------------- KDA
+def kda_checkpoint(layer: KDALayer, seed: int = 0) -> torch.Tensor:
+    """Initial fp32 checkpoint S[B, H, dv, dk] ~ N(0, state_std)."""
+    shape = (layer.batch, layer.nheads, layer.dv, layer.dk)
+    if layer.state_std == 0.0:
+        return torch.zeros(shape)
+    return torch.randn(shape, generator=_generator(seed, "kda.S0")) * layer.state_std
+
+
+def kda_tokens(layer: KDALayer, step: int, seed: int = 0):
+    """One decode token: q,k[B,H,dk], v[B,H,dv] (input dtype), alpha[B,H,dk] fp32 (one
+    gate per key channel, the GDN recipe drawn per channel), beta[B,H] fp32."""
+    B, H, dk, dv = layer.batch, layer.nheads, layer.dk, layer.dv
+    key = (seed, "kda.tok", int(step))
+    dt_ = torch_dtype(layer.dtype)
+    q = torch.randn((B, H, dk), generator=_generator(*key, "q"))
+    k = torch.randn((B, H, dk), generator=_generator(*key, "k"))
+    q = q / torch.linalg.vector_norm(q, dim=-1, keepdim=True)
+    k = k / torch.linalg.vector_norm(k, dim=-1, keepdim=True)
+    v = torch.randn((B, H, dv), generator=_generator(*key, "v"))
+    za = torch.randn((B, H, dk), generator=_generator(*key, "alpha"))
+    zb = torch.randn((B, H), generator=_generator(*key, "beta"))
+    return {"q": q.to(dt_), "k": k.to(dt_), "v": v.to(dt_),
+            "alpha": torch.exp(-0.1 * F.softplus(za)).float(), "beta": torch.sigmoid(zb).float()}
 
 
 # ------------------------------------------------------------------ branching
