@@ -298,7 +298,59 @@ class GDNWork:
         return time.perf_counter() - t0
 
 
-WORKLOADS = {"mamba2": Mamba2Work, "gdn": GDNWork}
+class KDAWork(GDNWork):
+    """Kimi Delta Attention layer (per-channel gates) of the GDN serving shape."""
+    name = "kda"
+    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/kda.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
+
+    def __init__(self, dev, seed, batch=None, read_fmt=0, window=None):
+        self.shape = s = si.KDA_SERVING if batch is None else si.KDA_SERVING.with_(batch=batch)
+        if window is not None:
+            self.shape = s = s.with_(window=window)
+        self.seed, self.dev, self.read_fmt = seed, dev, read_fmt
+        self.h0 = si.kda_checkpoint(s, seed).to(dev)
+        self.host_pool = [si.kda_tokens(s, t, seed) for t in range(POOL)]
+        self.pool = [[tok[k].to(dev) for k in self.keys] for tok in self.host_pool]
+        if dev.type == "cuda":
+            from hybrid_ssm_decode_replayssm_b200 import rssm
+            self.desc = rssm.make_desc(rssm.RSSM_KDA, s.batch, s.nheads, s.dv, s.dk, window=s.window,
+                                       max_draft=0, in_dtype=rssm.RSSM_BF16)
+        self.out_shape = (s.batch, s.nheads, s.dv)
+        self.tokens_per_call = s.batch
+        self.workload = (f"KDA decode layer: batch {s.batch}, {s.nheads} heads, d_k = d_v = {s.dk}, "
+                         f"bf16 q/k/v, fp32 per-channel alpha, fp32 beta, fp32 checkpoint, L={s.window}")
+
+    def bytes_per_call(self, pos):
+        """Algorithmic bytes of the decode call at window position pos (1..L)."""
+        s = self.shape
+        BH, dk, dv, L = s.batch * s.nheads, s.dk, s.dv, s.window
+        ck = BH * dv * dk * 4
+        inputs = BH * (2 * dk + dv) * 2 + BH * dk * 4 + BH * 4       # q, k, v, alpha per channel, beta
+        append = BH * (dk + dv) * 2 + BH * dk * 4 + BH * 4 + BH * dv * 4   # k, v, g, beta; new w
+        entry = BH * dk * 2 + BH * dk * 4 + BH * dv * 4               # k, g, w per window entry
+        out = BH * dv * 4
+        fold = ck if pos == L else 0
+        return ck + inputs + append + (pos - 1) * entry + out + fold
+
+    def conventional_bytes(self):
+        s = self.shape
+        BH = s.batch * s.nheads
+        return 2 * BH * s.dv * s.dk * 4 + BH * (2 * s.dk + s.dv) * 2 + BH * s.dk * 4 + BH * 4 + BH * s.dv * 4
+
+    def oracle_sample(self, nseq, steps, seed):
+        """Time the fp64 oracle (conventional KDA rule) on nseq sequences x all heads."""
+        from oracle import kda as ok
+        S = self.h0[:nseq].double().cpu().numpy()
+        toks = [{k: v[:nseq].double().numpy() for k, v in self.host_pool[t % POOL].items()} for t in range(steps)]
+        t0 = time.perf_counter()
+        for tok in toks:
+            S, _ = ok.step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+        return time.perf_counter() - t0
+
+
+WORKLOADS = {"mamba2": Mamba2Work, "gdn": GDNWork, "kda": KDAWork}
 
 
 # ------------------------------------------------------------------ timing
@@ -689,7 +741,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
-    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,speculative,read_copy,quantized_state,graph,branch",
+    ap.add_argument("--legs", default="replay,conventional,e2e,gdn,kda,speculative,read_copy,quantized_state,graph,branch",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -773,28 +825,31 @@ def main():
     gw = None
     if world == 1 and args.layer == "mamba2" and legs & {"gdn", "speculative", "read_copy", "quantized_state", "graph", "branch"}:
         gw = GDNWork(dev, seed, args.batch)
+    def layer_leg(w):
+        """Replay decode of another layer type at its serving shape, with its
+        conventional kernel timed beside it."""
+        wl = w.layer()
+        wout = torch.empty(w.out_shape, device=dev)
+        w_steps = max(20, args.steps // 3)
+        w_el, w_per, w_pos, _, _ = time_replay(w, wl, w_steps, args.warmup, L, wout, dev, 1, local)
+        w_bytes = sum(w.bytes_per_call(p) for p in w_pos)
+        wc_el = time_conventional(w, wl, w_steps, args.warmup, L, wout, 1)
+        res = {"workload": w.workload, "value": round(w.tokens_per_call * L * w_steps / w_el, 1),
+               "unit": "tokens/s", "hbm_gbs": round(w_bytes / w_el / 1e9, 1),
+               "roofline_frac": round(w_bytes / sum(w_per) / 1e9 / measured_peak()[0], 4),
+               "launch_us_fold": round(statistics.mean(p for p, q in zip(w_per, w_pos) if q == L) * 1e6, 2),
+               "launch_us_nofold": round(statistics.mean(p for p, q in zip(w_per, w_pos) if q != L) * 1e6, 2),
+               "conventional_tokens_per_s": round(w.tokens_per_call * L * w_steps / wc_el, 1),
+               "replay_speedup": round(wc_el / w_el, 3), "status_bits": wl.get_status()}
+        del wl
+        torch.cuda.empty_cache()
+        return res
+
     if world == 1 and "gdn" in legs and gw is not None:
-        gl = gw.layer()
-        gout = torch.empty(gw.out_shape, device=dev)
-        g_el, g_per, g_pos, _, _ = time_replay(gw, gl, max(20, args.steps // 3), args.warmup, L, gout, dev, 1, local)
-        g_steps = max(20, args.steps // 3)
-        g_bytes = sum(gw.bytes_per_call(p) for p in g_pos)
-        gc_el = time_conventional(gw, gl, g_steps, args.warmup, L, gout, 1)
-        extras["gdn"] = {"workload": gw.workload, "value": round(gw.tokens_per_call * L * g_steps / g_el, 1),
-                         "unit": "tokens/s", "hbm_gbs": round(g_bytes / g_el / 1e9, 1),
-                         "roofline_frac": round(g_bytes / sum(g_per) / 1e9 / measured_peak()[0], 4),
-                         "launch_us_fold": round(statistics.mean(p for p, q in zip(g_per, g_pos) if q == L) * 1e6, 2),
-                         "launch_us_nofold": round(statistics.mean(p for p, q in zip(g_per, g_pos) if q != L) * 1e6, 2),
-                         "conventional_tokens_per_s": round(gw.tokens_per_call * L * g_steps / gc_el, 1),
-                         "replay_speedup": round(gc_el / g_el, 3)}
-        del gl
+        extras["gdn"] = layer_leg(gw)
+    if world == 1 and "kda" in legs and args.layer == "mamba2":
+        extras["kda"] = layer_leg(KDAWork(dev, seed, args.batch))
         torch.cuda.empty_cache()
-    if world == 1 and "speculative" in legs:
-        extras["speculative"] = {"mamba2": speculative_leg(work)}
-        torch.cuda.empty_cache()
-        if gw is not None:
-            extras["speculative"]["gdn"] = speculative_leg(gw)
-            torch.cuda.empty_cache()
     if world == 1 and "branch" in legs:
         extras["branch"] = {"how": "beam-search-like: each sequence re-parented with probability 1/2 before "
                                    "every token", work.name: branch_leg(work)}

@@ -7,6 +7,7 @@
 #include <string>
 
 #include "rssm_internal.h"
+#include "rssm_kda.h"
 
 struct rssm_handle {
   rssm_layer_desc d;
@@ -48,8 +49,8 @@ bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 int validate_desc(const rssm_layer_desc *d) {
   if (!d) return fail(RSSM_ERR_INVALID_ARG, "desc is NULL");
-  if (d->kind != RSSM_MAMBA2 && d->kind != RSSM_GDN)
-    return fail(RSSM_ERR_INVALID_ARG, "kind must be RSSM_MAMBA2 or RSSM_GDN");
+  if (d->kind != RSSM_MAMBA2 && d->kind != RSSM_GDN && d->kind != RSSM_KDA)
+    return fail(RSSM_ERR_INVALID_ARG, "kind must be RSSM_MAMBA2, RSSM_GDN or RSSM_KDA");
   if (d->batch < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1)
     return fail(RSSM_ERR_INVALID_ARG, "batch, nheads, headdim and dstate must be positive");
   if ((long long)d->batch * d->nheads > (1LL << 31) - 1)
@@ -66,10 +67,13 @@ int validate_desc(const rssm_layer_desc *d) {
       d->read_fmt != RSSM_READ_NVFP4)
     return fail(RSSM_ERR_INVALID_ARG, "unknown read_fmt");
   const bool sup = d->kind == RSSM_MAMBA2 ? rssm::mamba2_supported(d->headdim, d->dstate)
-                                          : rssm::gdn_supported(d->headdim, d->dstate);
+                    : d->kind == RSSM_GDN  ? rssm::gdn_supported(d->headdim, d->dstate)
+                                           : rssm::kda_supported(d->headdim, d->dstate);
   if (!sup)
     return fail(RSSM_ERR_UNSUPPORTED, "no kernel for %s headdim=%d dstate=%d in this build",
-                d->kind == RSSM_MAMBA2 ? "Mamba-2" : "GDN", d->headdim, d->dstate);
+                d->kind == RSSM_MAMBA2 ? "Mamba-2" : d->kind == RSSM_GDN ? "GDN" : "KDA", d->headdim, d->dstate);
+  if (d->kind == RSSM_KDA && d->read_fmt != RSSM_READ_FP32)
+    return fail(RSSM_ERR_UNSUPPORTED, "KDA layers read the fp32 checkpoint (no read copy in this build)");
   return RSSM_OK;
 }
 
@@ -88,6 +92,12 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
     L->buf_off[0] = off; off = align256(off + B * H * cap * R * esz);      // x_buf
     L->buf_off[1] = off; off = align256(off + B * G * cap * C * esz);      // B_buf
     L->buf_off[2] = off; off = align256(off + B * H * cap * sizeof(float)); // dt_buf
+  } else if (d->kind == RSSM_KDA) {
+    L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf [B,H,cap,dk]
+    L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf [B,H,cap,dv]
+    L->buf_off[2] = off; off = align256(off + B * H * cap * C * sizeof(float)); // g_buf [B,H,cap,dk]
+    L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf [B,H,cap]
+    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf [B,H,cap,dv]
   } else {
     L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf [B,H,cap,dk]
     L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf [B,H,2,cap,dv/2]
@@ -149,7 +159,7 @@ rssm::StepArgs step_args(const rssm_handle *h, int mode, int m) {
   a.buf0 = h->buf + h->lay.buf_off[0];
   a.buf1 = h->buf + h->lay.buf_off[1];
   a.buf2 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[2]);
-  if (d.kind == RSSM_GDN) {
+  if (d.kind != RSSM_MAMBA2) {
     a.buf3 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[3]);
     a.buf4 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[4]);
   }
@@ -190,6 +200,14 @@ int plan_slots_for(rssm_handle *h, const rssm::StepArgs &a, cudaStream_t s) {
   return RSSM_OK;
 }
 
+cudaError_t replay_launch(const rssm_handle *h, const rssm::StepArgs &a, cudaStream_t s) {
+  switch (h->d.kind) {
+    case RSSM_MAMBA2: return rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, s);
+    case RSSM_GDN: return rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, s);
+    default: return rssm::kda_step(a, h->d.in_dtype, s);
+  }
+}
+
 int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *out,
                 const int32_t *mask, cudaStream_t s) {
   rssm::StepArgs a = step_args(h, mode, m);
@@ -199,8 +217,7 @@ int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *ou
   a.mask = mask;
   int rc = plan_slots_for(h, a, s);
   if (rc) return rc;
-  cudaError_t e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, s)
-                                           : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, s);
+  cudaError_t e = replay_launch(h, a, s);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");
   return ok();
@@ -284,6 +301,7 @@ int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev, rssm_
 
 int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.kind == RSSM_KDA) return fail(RSSM_ERR_UNSUPPORTED, "verify is not built for KDA layers");
   if (h->d.max_draft < 1) return fail(RSSM_ERR_STATE, "handle was created with max_draft = 0");
   if (k < 1 || k > h->d.max_draft)
     return fail(RSSM_ERR_CAPACITY, "k = %d outside [1, max_draft = %d]", k, h->d.max_draft);
@@ -345,7 +363,9 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev, float *sta
   a.out = static_cast<float *>(out_dev);
   cudaError_t e = h->d.kind == RSSM_MAMBA2
                       ? rssm::mamba2_conventional(a, h->d.in_dtype, RSSM_READ_FP32, (cudaStream_t)stream)
-                      : rssm::gdn_conventional(a, h->d.in_dtype, RSSM_READ_FP32, (cudaStream_t)stream);
+                  : h->d.kind == RSSM_GDN
+                      ? rssm::gdn_conventional(a, h->d.in_dtype, RSSM_READ_FP32, (cudaStream_t)stream)
+                      : rssm::kda_conventional(a, h->d.in_dtype, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "conventional kernel launch");
   return ok();
@@ -413,6 +433,11 @@ int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream)
     const int outer[3] = {H, d.ngroups, H}, entry[3] = {d.headdim * esz, d.dstate * esz, 4};
     b.nreg = 3;
     for (int r = 0; r < 3; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
+  } else if (d.kind == RSSM_KDA) {   // k [H][cap][dk] | v [H][cap][dv] | g [H][cap][dk] fp32 | beta | w
+    const int outer[5] = {H, H, H, H, H};
+    const int entry[5] = {d.dstate * esz, d.headdim * esz, d.dstate * 4, 4, d.headdim * 4};
+    b.nreg = 5;
+    for (int r = 0; r < 5; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
   } else {   // k [H][cap][dk] | v [2H][cap][dv/2] | g, beta [H][cap] | w [2H][cap][dv/2] fp32
     const int outer[5] = {H, 2 * H, H, H, 2 * H};
     const int entry[5] = {d.dstate * esz, d.headdim / 2 * esz, 4, 4, d.headdim / 2 * 4};
@@ -542,8 +567,7 @@ extern "C" int rssm_decode_step_static_scratch(rssm_handle *h, const void *const
   a.arrivals = arrivals;
   rc = plan_slots_for(h, a, (cudaStream_t)stream);
   if (rc) return rc;
-  e = h->d.kind == RSSM_MAMBA2 ? rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream)
-                               : rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, (cudaStream_t)stream);
+  e = replay_launch(h, a, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");
   return ok();

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(HERE, "librssm.so")
 RSSM_OK, RSSM_ERR_INVALID_ARG, RSSM_ERR_UNSUPPORTED = 0, 1, 2
 RSSM_ERR_CAPACITY, RSSM_ERR_STATE, RSSM_ERR_CUDA, RSSM_ERR_TIMEOUT = 3, 4, 5, 6
 RSSM_STATUS_CAPACITY, RSSM_STATUS_STATE = 1, 2
-RSSM_MAMBA2, RSSM_GDN = 1, 2
+RSSM_MAMBA2, RSSM_GDN, RSSM_KDA = 1, 2, 3
 RSSM_F32, RSSM_BF16 = 0, 1
 RSSM_READ_FP32, RSSM_READ_FP8_E4M3_ROW, RSSM_READ_NVFP4 = 0, 1, 2
 

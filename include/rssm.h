@@ -74,7 +74,7 @@ enum {
   RSSM_STATUS_TIMEOUT = 1u << 2   /* a bounded wait for an asynchronous copy gave up   */
 };
 
-enum { RSSM_MAMBA2 = 1, RSSM_GDN = 2 };
+enum { RSSM_MAMBA2 = 1, RSSM_GDN = 2, RSSM_KDA = 3 };
 enum { RSSM_F32 = 0, RSSM_BF16 = 1 };
 enum {
   RSSM_READ_FP32 = 0,        /* reads come from the fp32 checkpoint itself      */
@@ -88,10 +88,14 @@ enum {
  *            input group h / (nheads / ngroups).
  *   GDN:     state S [batch, nheads, headdim (= d_v), dstate (= d_k)] fp32,
  *            mapping keys to values; ngroups is ignored.
+ *   KDA:     as GDN, with one gate per key channel (Kimi Delta Attention,
+ *            named by [teaser]; read as S <- S Diag(alpha) (I - beta k k^T)
+ *            + beta v k^T, o = out_scale S q): replay decode and flush on the
+ *            fp32 checkpoint; no read copy, no verify in this build.
  * A "row" of the state is its last dimension: the contraction vector of one
  * output element (h[b,h,p,:] or S[b,h,i,:]).
  * Supported by this build: Mamba-2 headdim 64 with dstate 64 or 128;
- * GDN headdim = dstate = 128; 1 <= window <= 32; 0 <= max_draft <= 8 and
+ * GDN and KDA headdim = dstate = 128; 1 <= window <= 32; 0 <= max_draft <= 8 and
  * max_draft <= window.
  */
 typedef struct {
@@ -120,6 +124,9 @@ typedef struct {
  *                 g_buf [B,H,cap] fp32 (ln alpha) | beta_buf [B,H,cap] fp32 |
  *                 w_buf [B,H,2,cap,dv/2] fp32 (solved w_s, half-major; a cache
  *                 for reads, never used by a fold)
+ *   buf, KDA:     k_buf [B,H,cap,dk] in_dtype | v_buf [B,H,cap,dv] in_dtype |
+ *                 g_buf [B,H,cap,dk] fp32 (ln alpha per channel) |
+ *                 beta_buf [B,H,cap] fp32 | w_buf [B,H,cap,dv] fp32 (solved w_s)
  *   read copy, FP8 row: codes [B,H,R,C] uint8 | scales [B,H,R] fp32
  *   read copy, NVFP4:   codes [B,H,R,C/2] uint8 (element 2i in the low
  *                       nibble) | scales [B,H,R,C/16] uint8 (E4M3)
@@ -190,6 +197,7 @@ int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev);
  *            (in_dtype; dt already softplus'd);
  *   GDN:     in[0] q [B,H,dk], in[1] k [B,H,dk], in[2] v [B,H,dv] (in_dtype),
  *            in[3] alpha [B,H], in[4] beta [B,H] (fp32).
+ *   KDA:     as GDN with in[3] alpha [B,H,dk] (fp32, one gate per key channel).
  * out_dev: fp32 y [B,H,P] / o [B,H,dv].
  * With auto_flush: a row whose window is already full is folded first, and a
  * row whose window becomes full (len == L) is folded after its output is
@@ -207,6 +215,7 @@ int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev,
  * with a draft axis after the batch axis ([B,k,...]); out_dev is [B,k,H,P] /
  * [B,k,H,dv].  Output j is the output after drafts 0..j.  1 <= k <= max_draft.
  * A row with len + k > L is folded first (auto_flush; else CAPACITY, skipped).
+ * KDA layers: RSSM_ERR_UNSUPPORTED.
  */
 int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev,
                 rssm_stream_t stream);

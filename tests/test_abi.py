@@ -196,3 +196,26 @@ def test_branch_calls_check_arguments():
         assert L.rssm_get_slots(h, None, None) == rssm.RSSM_ERR_INVALID_ARG
     finally:
         L.rssm_destroy(h)
+
+
+def test_kda_descriptor_and_layout():
+    base = dict(kind=rssm.RSSM_KDA, batch=2, nheads=4, headdim=128, dstate=128, window=8, max_draft=0)
+    code, (ck, buf, rc, meta), lay = _sizes(_desc(**base))
+    assert code == rssm.RSSM_OK and rc == 0 and ck == 2 * 4 * 128 * 128 * 4
+    B, H, cap, d = 2, 4, 9, 128
+    assert lay.cap == cap
+    assert lay.buf_off[1] >= B * H * cap * d * 2                       # k ring (bf16)
+    assert lay.buf_off[3] - lay.buf_off[2] >= B * H * cap * d * 4      # per-channel log gates (fp32)
+    assert buf >= lay.buf_off[4] + B * H * cap * d * 4                 # w rows (fp32)
+    assert _sizes(_desc(**dict(base, read_fmt=rssm.RSSM_READ_NVFP4)))[0] == rssm.RSSM_ERR_UNSUPPORTED
+    assert _sizes(_desc(**dict(base, headdim=64)))[0] == rssm.RSSM_ERR_UNSUPPORTED
+    L = rssm.lib()
+    fake = 1 << 20
+    h = C.c_void_p()
+    d_ = _desc(**dict(base, max_draft=2))
+    assert L.rssm_create(C.byref(d_), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        ins = (C.c_void_p * 5)(fake, fake, fake, fake, fake)
+        assert L.rssm_verify(h, 1, ins, fake, None) == rssm.RSSM_ERR_UNSUPPORTED
+    finally:
+        L.rssm_destroy(h)

@@ -1,0 +1,109 @@
+"""Kimi Delta Attention on the GPU against the fp64 oracle (oracle.kda).
+
+KDA is the third SSM layer type the pages name ("ReplaySSM: Rethinking State
+Storage for Faster Hybrid-Model Decoding", babnews.org teaser); it is read as
+the gated delta rule with one gate per key channel.  The replay kernel keeps
+the fp32 checkpoint plus a window of inputs and cached w rows, folds the
+window when it fills, and must give the recurrence's outputs and states:
+
+* every output and the checkpoint after every fold, fp32 inputs (1e-4) over
+  window lengths 1..32 and bf16 inputs (2e-3);
+* the conventional per-token kernel (the in-run baseline) against the oracle;
+* explicit masked flush, restore to a position, and branching (rows sharing
+  checkpoint slots) against the oracle's window rules;
+* verify is not built for KDA and says so.
+"""
+import numpy as np
+import pytest
+import torch
+
+import seeded_inputs as si
+from gpu_common import DEV, KDA_KEYS, assert_close, dev_inputs, kda_layer, to64, tok64
+from hybrid_ssm_decode_replayssm_b200 import rssm
+from oracle import branch as ob
+from oracle import kda as ok
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-3}
+
+
+def _step(S, tok):
+    return ok.step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+
+
+@pytest.mark.parametrize("L,dtype", [(1, "f32"), (4, "f32"), (16, "f32"), (32, "f32"), (16, "bf16")])
+def test_decode_and_folds_against_oracle(L, dtype):
+    shape = si.KDALayer(batch=3, nheads=4, dk=128, dv=128, window=L, dtype=dtype, state_std=0.05)
+    layer, S0 = kda_layer(shape)
+    S = to64(S0)
+    out = torch.empty((3, 4, 128), device=DEV)
+    T = max(40, 2 * L + 3)
+    ck = S.copy()
+    for t in range(T):
+        tok = si.kda_tokens(shape, t, seed=2)
+        layer.decode_step(dev_inputs(tok, KDA_KEYS), out)
+        S, y = _step(S, tok64(tok))
+        assert_close(out.cpu(), y, TOL[dtype], f"L={L} step {t}: output")
+        if (t + 1) % L == 0:
+            ck = S.copy()
+        if t % 7 == 0 or (t + 1) % L == 0:
+            assert_close(layer.ckpt.cpu(), ck, TOL[dtype], f"L={L} step {t}: checkpoint")
+    layer.flush()
+    assert_close(layer.ckpt.cpu(), S, TOL[dtype], "checkpoint after the final flush")
+    assert layer.get_status() == 0
+
+
+def test_conventional_kernel_against_oracle():
+    shape = si.KDALayer(batch=4, nheads=8, dk=128, dv=128, window=16, dtype="bf16", state_std=0.05)
+    layer, S0 = kda_layer(shape)
+    state = S0.to(DEV).contiguous()
+    out = torch.empty((4, 8, 128), device=DEV)
+    S = to64(S0)
+    for t in range(6):
+        tok = si.kda_tokens(shape, t, seed=3)
+        layer.conventional_step(state, state, dev_inputs(tok, KDA_KEYS), out)
+        S, y = _step(S, tok64(tok))
+        assert_close(out.cpu(), y, TOL["bf16"], f"conventional y step {t}")
+    assert_close(state.cpu(), S, TOL["bf16"], "conventional state")
+
+
+def test_flush_restore_branch_against_oracle():
+    shape = si.KDALayer(batch=6, nheads=4, dk=128, dv=128, window=4, dtype="bf16", state_std=0.05)
+    layer, S0 = kda_layer(shape, branching=True)
+    rows = ob.BranchingRows(to64(S0), 4, layer.layout.cap, _step)
+    out = torch.empty((6, 4, 128), device=DEV)
+    rng = np.random.default_rng(3)
+    ops = ["decode", "decode", "branch", "decode", "restore", "decode", "decode", "flush", "decode",
+           "branch", "decode", "decode", "decode", "restore", "decode", "decode", "decode", "decode"]
+    for i, op in enumerate(ops):
+        if op == "decode":
+            tok = si.kda_tokens(shape, i, seed=5)
+            layer.decode_step(dev_inputs(tok, KDA_KEYS), out)
+            y = rows.decode(tok64(tok))
+            assert_close(out.cpu(), y, TOL["bf16"], f"{op} {i}")
+        elif op == "branch":
+            parent = si.branch_parents(6, i, seed=2).numpy()
+            layer.branch(torch.from_numpy(parent).to(DEV))
+            rows.branch(parent)
+        elif op == "restore":
+            keep = [int(rng.integers(0, n + 1)) for n in rows.book.len]
+            layer.restore(torch.tensor(keep, dtype=torch.int32, device=DEV))
+            rows.restore(keep)
+        else:
+            mask = [1, 1, 0, 1, 0, 1]
+            layer.flush(torch.tensor(mask, dtype=torch.int32, device=DEV))
+            rows.flush(mask)
+        assert layer.get_status(clear=True) == 0, f"{op} {i}: status"
+        bk = [list(map(int, r)) for r in layer.get_bookkeeping().cpu().numpy()]
+        assert bk == [list(x) for x in rows.book.snapshot()], f"{op} {i}: pointers"
+        assert_close(layer.checkpoint_rows().cpu(), rows.checkpoint(), TOL["bf16"], f"{op} {i}: checkpoints")
+
+
+def test_verify_is_not_built_for_kda():
+    shape = si.KDALayer(batch=2, nheads=4, dk=128, dv=128, window=8, dtype="bf16")
+    layer, _ = kda_layer(shape)
+    tok = si.kda_tokens(shape, 0)
+    with pytest.raises(rssm.RSSMError) as e:
+        layer.verify(1, dev_inputs(tok, KDA_KEYS), torch.empty((2, 1, 4, 128), device=DEV))
+    assert e.value.code == rssm.RSSM_ERR_UNSUPPORTED
