@@ -850,6 +850,12 @@ def main():
     if world == 1 and "kda" in legs and args.layer == "mamba2":
         extras["kda"] = layer_leg(KDAWork(dev, seed, args.batch))
         torch.cuda.empty_cache()
+    if world == 1 and "speculative" in legs:
+        extras["speculative"] = {"mamba2": speculative_leg(work)}
+        torch.cuda.empty_cache()
+        if gw is not None:
+            extras["speculative"]["gdn"] = speculative_leg(gw)
+            torch.cuda.empty_cache()
     if world == 1 and "branch" in legs:
         extras["branch"] = {"how": "beam-search-like: each sequence re-parented with probability 1/2 before "
                                    "every token", work.name: branch_leg(work)}

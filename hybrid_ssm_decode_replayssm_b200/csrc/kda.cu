@@ -85,10 +85,52 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   float *qv = dec + wmax * KD, *vv = qv + KD, *eG = vv + KD, *uu = eG + KD, *yy = uu + KD;
   float *Adot = yy + KD, *Bdot = Adot + wmax;   // window dot products
 
+  // the checkpoint tile is requested first: its address needs nothing but the
+  // sequence's slot (b itself unless the layer branches)
+  const int row0 = warp * kRowsPerWarp, c0 = lane * 4;
+  const int src_slot = a.slot ? a.slot[b] : b;
+  const float *src = a.hc + ((size_t)src_slot * a.H + h) * KD * KD;
+  float4 S[kRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) S[i] = ld_stream(src + (size_t)(row0 + i) * KD + c0);
+  // and the new token's inputs (thread c < KD: channel / value row c)
+  Tin kr{}, vr{}, qr{};
+  float ar = 1.0f;
+  if (a.m == 1 && tid < KD) {
+    kr = reinterpret_cast<const Tin *>(a.in[1])[(size_t)bh * KD + tid];
+    vr = reinterpret_cast<const Tin *>(a.in[2])[(size_t)bh * KD + tid];
+    qr = reinterpret_cast<const Tin *>(a.in[0])[(size_t)bh * KD + tid];
+    ar = reinterpret_cast<const float *>(a.in[3])[(size_t)bh * KD + tid];
+  }
+
   const RowPlan rp = plan_row(a, b);
   if (rp.refuse) {
     if (rp.bit && h == 0 && tid == 0) atomicOr(a.status, rp.bit);
     return;
+  }
+  // Every CTA of sequence b has read its pointers once all of them have counted
+  // in, so the last to count in moves them now (its own threads have read them:
+  // the barrier below), off the end of the kernel.
+  __syncthreads();
+  if (tid == 0 && atomicAdd(a.arrivals + b, 1) == a.H - 1) {
+    a.arrivals[b] = 0;
+    int st2 = rp.st, n2 = rp.n, fl = a.flushes[b];
+    if (rp.pre) {
+      st2 = (rp.st + rp.n) % a.cap;
+      n2 = 0;
+      ++fl;
+    }
+    if (a.mode == kDecode) {
+      n2 += 1;
+      if (rp.post) {
+        st2 = (st2 + n2) % a.cap;
+        n2 = 0;
+        ++fl;
+      }
+    }
+    a.start[b] = st2;
+    a.len[b] = n2;
+    a.flushes[b] = fl;
   }
   const int m = a.m, st = rp.st;
   int n = rp.n;
@@ -100,13 +142,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   float *bring = a.buf3 + (size_t)bh * cap;
   float *wring = a.buf4 + (size_t)bh * cap * KD;
 
-  // state tile: rows row0 .. row0+15, columns c0 .. c0+3 (streamed, evict-first)
-  const int row0 = warp * kRowsPerWarp, c0 = lane * 4;
-  const float *src = a.hc + ((size_t)rp.src * a.H + h) * KD * KD;
-  float *dst = a.hc + ((size_t)rp.dst * a.H + h) * KD * KD;
-  float4 S[kRowsPerWarp];
-#pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) S[i] = ld_stream(src + (size_t)(row0 + i) * KD + c0);
+  float *dst = a.hc + ((size_t)rp.dst * a.H + h) * KD * KD;   // where a fold writes
 
   // committed window rows into shared memory
   for (int idx = tid; idx < n * KD; idx += kKdaThreads) {
@@ -138,17 +174,12 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
     // ---- the new token: entry t = n of the window, ring slot (st_new + n) % cap
     const int t = n;
     const size_t slot = (size_t)((st_new + t) % cap);
-    const Tin *qin = reinterpret_cast<const Tin *>(a.in[0]) + (size_t)bh * KD;
-    const Tin *kin = reinterpret_cast<const Tin *>(a.in[1]) + (size_t)bh * KD;
-    const Tin *vin = reinterpret_cast<const Tin *>(a.in[2]) + (size_t)bh * KD;
-    const float *ain = reinterpret_cast<const float *>(a.in[3]) + (size_t)bh * KD;
     const float beta = reinterpret_cast<const float *>(a.in[4])[bh];
     if (tid < KD) {
-      const Tin kr = kin[tid], vr = vin[tid];
-      const float g = logf(ain[tid]);
+      const float g = logf(ar);
       kw[t * KD + tid] = to_f32<Tin>(kr);
       gw[t * KD + tid] = g;
-      qv[tid] = to_f32<Tin>(qin[tid]);
+      qv[tid] = to_f32<Tin>(qr);
       vv[tid] = to_f32<Tin>(vr);
       kring_w[slot * KD + tid] = kr;
       vring[slot * KD + tid] = vr;
@@ -211,32 +242,6 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
     } else if (pre) {
 #pragma unroll
       for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
-    }
-  }
-
-  // ---- the last CTA of sequence b moves its pointers
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(a.arrivals + b, 1) == a.H - 1) {
-      a.arrivals[b] = 0;
-      int st2 = st, n2 = rp.n, fl = a.flushes[b];
-      if (pre) {
-        st2 = (st + rp.n) % cap;
-        n2 = 0;
-        ++fl;
-      }
-      if (a.mode == kDecode) {
-        n2 += 1;
-        if (post) {
-          st2 = (st2 + n2) % cap;
-          n2 = 0;
-          ++fl;
-        }
-      }
-      a.start[b] = st2;
-      a.len[b] = n2;
-      a.flushes[b] = fl;
     }
   }
 }
