@@ -15,7 +15,7 @@
  *   - the checkpoint stays high precision for the recurrence while a
  *     low-precision (NVFP4) copy serves the reads [summary ¶4];
  *   - window L = 16 is the default [summary ¶6];
- *   - Mamba-2 and Gated DeltaNet are the SSM layers [teaser].
+ *   - Mamba-2, Gated DeltaNet and KDA are the SSM layers [teaser].
  * The pages print no formula.  The library implements the Mamba-2 and gated
  * delta-rule recurrences (Mamba-2 SSD; gated delta rule) in replay form:
  *   Mamba-2 (a_r = dt_r * A_h, seg(s,t) = sum_{s<r<=t} a_r, G_t = seg(0,t)):
@@ -25,6 +25,10 @@
  *     w_t = beta_t (v_t - e^{G_t} u_t - sum_{s<t} e^{seg(s,t)} (k_s . k_t) w_s)
  *     o_t = out_scale (e^{G_t} h_c q_t + sum_{s<=t} e^{seg(s,t)} (k_s . q_t) w_s)
  *     flush: h_c <- e^{G_l} h_c + sum_{s<=l} e^{seg(s,l)} w_s k_s^T
+ *   KDA (one gate per key channel, a_r = ln alpha_r elementwise, e^{.} and
+ *   (.) elementwise): as GDN with e^{G_t} u_t -> h_c (e^{G_t} (.) k_t),
+ *   (k_s . k_t) e^{seg} -> (k_s (.) e^{seg(s,t)}) . k_t, likewise for q_t, and
+ *     flush: h_c <- h_c Diag(e^{G_l}) + sum_{s<=l} w_s (k_s (.) e^{seg(s,l)})^T
  * which equal the token-by-token recurrences exactly (up to rounding).
  *
  * Conventions for every call
