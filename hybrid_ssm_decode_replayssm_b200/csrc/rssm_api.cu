@@ -477,6 +477,59 @@ int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
   return ok();
 }
 
+// A layer's whole replay state as one host blob: checkpoint (all slots) | read
+// copy | ring regions (not the branch scratch) | meta.
+namespace {
+struct Piece {
+  uint8_t *dev;
+  size_t bytes;
+};
+int state_pieces(const rssm_handle *h, Piece (&p)[4]) {
+  p[0] = {reinterpret_cast<uint8_t *>(h->ckpt), h->ckpt_bytes};
+  p[1] = {h->rc, h->rc ? h->rc_bytes : 0};
+  p[2] = {h->buf, h->d.branching ? h->lay.branch_scratch_off : h->buf_bytes};
+  p[3] = {h->meta, h->meta_bytes};
+  return 4;
+}
+}  // namespace
+
+int rssm_state_bytes(rssm_handle *h, size_t *bytes) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!bytes) return fail(RSSM_ERR_INVALID_ARG, "bytes is NULL");
+  Piece p[4];
+  size_t total = 0;
+  for (int i = 0; i < state_pieces(h, p); ++i) total += p[i].bytes;
+  *bytes = total;
+  return ok();
+}
+
+static int copy_state(rssm_handle *h, uint8_t *host, size_t bytes, bool to_host, cudaStream_t s) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!host) return fail(RSSM_ERR_INVALID_ARG, "host buffer is NULL");
+  Piece p[4];
+  const int n = state_pieces(h, p);
+  size_t total = 0;
+  for (int i = 0; i < n; ++i) total += p[i].bytes;
+  if (bytes != total) return fail(RSSM_ERR_INVALID_ARG, "host buffer has %zu bytes, the state has %zu", bytes, total);
+  size_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    if (p[i].bytes == 0) continue;
+    cudaError_t e = to_host ? cudaMemcpyAsync(host + off, p[i].dev, p[i].bytes, cudaMemcpyDeviceToHost, s)
+                            : cudaMemcpyAsync(p[i].dev, host + off, p[i].bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, to_host ? "state export copy" : "state import copy");
+    off += p[i].bytes;
+  }
+  return ok();
+}
+
+int rssm_export_state(rssm_handle *h, void *host_dst, size_t bytes, rssm_stream_t stream) {
+  return copy_state(h, static_cast<uint8_t *>(host_dst), bytes, true, (cudaStream_t)stream);
+}
+
+int rssm_import_state(rssm_handle *h, const void *host_src, size_t bytes, rssm_stream_t stream) {
+  return copy_state(h, static_cast<uint8_t *>(const_cast<void *>(host_src)), bytes, false, (cudaStream_t)stream);
+}
+
 int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!out_dev) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");

@@ -34,6 +34,7 @@ EXPORTED = [
     "rssm_get_status", "rssm_last_error_string", "rssm_launch_count",
     "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
     "rssm_branch", "rssm_restore", "rssm_get_slots",
+    "rssm_state_bytes", "rssm_export_state", "rssm_import_state",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -85,6 +86,9 @@ def lib():
         L.rssm_branch.argtypes = [vp, vp, vp]
         L.rssm_restore.argtypes = [vp, vp, vp]
         L.rssm_get_slots.argtypes = [vp, vp, vp]
+        L.rssm_state_bytes.argtypes = [vp, C.POINTER(sz)]
+        L.rssm_export_state.argtypes = [vp, vp, sz, vp]
+        L.rssm_import_state.argtypes = [vp, vp, sz, vp]
         L.rssm_get_status.argtypes = [vp, C.POINTER(C.c_uint32), i32, vp]
         for name in EXPORTED:
             getattr(L, name).restype = C.c_int
@@ -242,6 +246,24 @@ class ReplayLayer:
         if not self.desc.branching:
             return self.ckpt.clone()
         return self.ckpt.index_select(0, self.get_slots(stream).long())
+
+    def state_bytes(self) -> int:
+        n = C.c_size_t()
+        check(lib().rssm_state_bytes(self.handle, C.byref(n)))
+        return n.value
+
+    def export_state(self, host=None, stream=None) -> torch.Tensor:
+        """The layer's whole replay state into a pinned host uint8 tensor (synchronised)."""
+        n = self.state_bytes()
+        if host is None:
+            host = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+        check(lib().rssm_export_state(self.handle, host.data_ptr(), n, _stream(stream)))
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+        return host
+
+    def import_state(self, host, stream=None):
+        check(lib().rssm_import_state(self.handle, host.data_ptr(), host.numel(), _stream(stream)))
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
 
     def get_bookkeeping(self, stream=None) -> torch.Tensor:
         out = torch.empty((4, self.desc.batch), dtype=torch.int32, device=self.ckpt.device)

@@ -340,6 +340,22 @@ int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream);
  * RSSM_ERR_STATE if the handle was created with branching = 0. */
 int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream);
 
+/*
+ * State export / import to host (serving-side preemption, migration between
+ * processes or GPUs).  The blob is the layer's whole replay state in one host
+ * buffer: checkpoint (every slot) | read copy | ring buffers | meta (pointers,
+ * slots, status), in that order, raw bytes; rssm_state_bytes gives its size.
+ * Import requires a handle created from the same descriptor.  Both are plain
+ * cudaMemcpyAsync calls on `stream` (pinned host memory makes them
+ * asynchronous; the caller synchronises before reading or reusing the blob).
+ * No kernel runs and nothing is converted: export then import is bit-exact.
+ * Errors: RSSM_ERR_INVALID_ARG for NULL pointers or a size that differs from
+ * rssm_state_bytes.
+ */
+int rssm_state_bytes(rssm_handle *h, size_t *bytes);
+int rssm_export_state(rssm_handle *h, void *host_dst, size_t bytes, rssm_stream_t stream);
+int rssm_import_state(rssm_handle *h, const void *host_src, size_t bytes, rssm_stream_t stream);
+
 /* Copy the per-sequence pointers into out_dev (device int32 [4, B]: start,
  * len, pending, flushes). */
 int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev,

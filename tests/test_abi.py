@@ -219,3 +219,25 @@ def test_kda_descriptor_and_layout():
         assert L.rssm_verify(h, 1, ins, fake, None) == rssm.RSSM_ERR_UNSUPPORTED
     finally:
         L.rssm_destroy(h)
+
+
+def test_state_io_checks_sizes():
+    """rssm_state_bytes = checkpoint + read copy + ring buffers + meta (branch scratch
+    excluded); export/import refuse a buffer of another size before any copy."""
+    L = rssm.lib()
+    fake = 1 << 20
+    for kw in ({}, {"read_fmt": rssm.RSSM_READ_NVFP4, "branching": True}):
+        d = _desc(**kw)
+        code, (ck, buf, rc, meta), lay = _sizes(d)
+        h = C.c_void_p()
+        assert L.rssm_create(C.byref(d), fake, fake, fake, fake, C.byref(h)) == rssm.RSSM_OK
+        try:
+            n = C.c_size_t()
+            assert L.rssm_state_bytes(h, C.byref(n)) == rssm.RSSM_OK
+            ring = lay.branch_scratch_off if kw.get("branching") else buf
+            assert n.value == ck + rc + ring + meta
+            assert L.rssm_export_state(h, fake, n.value + 1, None) == rssm.RSSM_ERR_INVALID_ARG
+            assert L.rssm_import_state(h, None, n.value, None) == rssm.RSSM_ERR_INVALID_ARG
+            assert L.rssm_state_bytes(h, None) == rssm.RSSM_ERR_INVALID_ARG
+        finally:
+            L.rssm_destroy(h)
