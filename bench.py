@@ -747,15 +747,22 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
-    rank, world, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
+    if args.impl == "reference":
+        # The oracle runs on the host cores: no GPU and no process group; under
+        # torchrun rank 0 alone runs it and the other ranks exit without work.
+        rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+        if world != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
+        local, dev = 0, torch.device("cpu")
+        if rank != 0:
+            return
+    else:
+        rank, world, local = dist_setup(args.gpus)
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
     seed = args.seed + rank
     legs = set(args.legs.split(","))
-    if args.impl == "reference":   # the oracle runs on the host: build the workload there
-        work = WORKLOADS[args.layer](torch.device("cpu"), seed, args.batch)
-    else:
-        work = WORKLOADS[args.layer](dev, seed, args.batch)
+    work = WORKLOADS[args.layer](dev, seed, args.batch)
     L = work.shape.window
     tokens_per_step = work.tokens_per_call * L
     cfg = {"workload": work.workload, "global_batch": work.shape.batch * world,
@@ -775,8 +782,6 @@ def main():
                     "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                             "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
-        if world > 1:
-            torch.distributed.destroy_process_group()
         return
 
     layer = work.layer()
