@@ -107,3 +107,83 @@ def test_nvfp4_quantiser_error_bound():
     ok = np.where(sval[..., None] == 0, np.abs(rows.reshape(32, 8, 16)) < 1e-5, err <= bound * 1.0001)
     assert ok.all()
 
+
+
+# ---- the scale rules themselves.  The bounds above hold for a range of
+#      divisors; these pin the divisor: the block / row maximum must land on the
+#      top code of the element format, within one rounding of the scale and
+#      never saturating beyond it, and data that already sits on a scaled code
+#      grid must come back exactly.
+
+def _blocks_with_spread(rng, nrows, ncols):
+    """Rows whose 16-element blocks have maxima spread over [0.1, 2000] (E4M3
+    block scales amax/6 stay normal: >= 2^-6 and <= 448)."""
+    rows = rng.standard_normal((nrows, ncols))
+    blocks = rows.reshape(nrows, ncols // 16, 16)
+    target = np.exp(rng.uniform(np.log(0.1), np.log(2000.0), size=blocks.shape[:2]))
+    blocks *= (target / np.max(np.abs(blocks), axis=-1))[..., None]
+    return blocks.reshape(nrows, ncols).astype(np.float32)
+
+
+def test_nvfp4_block_max_takes_top_code_without_saturating():
+    """s = E4M3(amax / 6): the block max divided by the decoded scale lies within
+    one E4M3 rounding (2^-4 relative) of 6, i.e. in [6 / (1 + 2^-4), 6 / (1 - 2^-4)],
+    so it encodes to magnitude code 7 (6.0) and nothing saturates by more than
+    that rounding.  A divisor of 4 or 8 (or 5.5, 6.5) fails one of the bounds."""
+    rng = np.random.default_rng(11)
+    rows = _blocks_with_spread(rng, 256, 128)
+    codes, sc = codecs.nvfp4_quantize(rows)
+    sval = codecs.e4m3_decode(sc).astype(np.float32)
+    blk = rows.reshape(256, 8, 16)
+    q = (blk / sval[..., None]).astype(np.float32)                  # the quantiser's own fp32 division
+    qmax = np.max(np.abs(q), axis=-1)
+    assert np.all(qmax <= np.float32(6.0 / (1 - 2.0 ** -4)) * (1 + 2.0 ** -22))
+    assert np.all(qmax >= np.float32(6.0 / (1 + 2.0 ** -4)) * (1 - 2.0 ** -22))
+    arg = np.argmax(np.abs(blk), axis=-1)
+    top = np.take_along_axis(codes.reshape(256, 8, 16), arg[..., None], axis=-1)[..., 0]
+    assert np.all((top & 0x7) == 0x7)
+    assert np.all(((top >> 3) & 1) == np.signbit(np.take_along_axis(blk, arg[..., None], -1)[..., 0]))
+
+
+def test_nvfp4_exact_on_scaled_e2m1_grid():
+    """Blocks of E2M1 values times 2^e whose max is 6 * 2^e have scale exactly 2^e
+    (E4M3-representable for -6 <= e <= 8), so they quantise without error."""
+    rng = np.random.default_rng(12)
+    grid = np.concatenate([codecs.E2M1_VALUES, -codecs.E2M1_VALUES])
+    for e in range(-6, 9):
+        blocks = rng.choice(grid, size=(64, 16))
+        blocks[np.arange(64), rng.integers(0, 16, 64)] = rng.choice([6.0, -6.0], 64)
+        rows = (blocks * 2.0 ** e).reshape(8, 128).astype(np.float32)
+        codes, sc = codecs.nvfp4_quantize(rows)
+        np.testing.assert_array_equal(codecs.e4m3_decode(sc), 2.0 ** e)
+        np.testing.assert_array_equal(codecs.nvfp4_dequantize(codes, sc), rows)
+
+
+def test_fp8_row_max_takes_top_code_without_saturating():
+    """s = amax / 448 (fp32): the row max divided by s is 448 up to fp32 rounding,
+    so it encodes to 0x7E (0xFE when negative) and no element saturates beyond
+    one rounding of the scale.  Divisors such as 430 or 470 fail."""
+    rng = np.random.default_rng(13)
+    rows = rng.standard_normal((512, 128)) * np.exp(rng.uniform(-12, 12, size=(512, 1)))
+    rows = rows.astype(np.float32)
+    codes, s = codecs.fp8_row_quantize(rows)
+    q = (rows / s[:, None]).astype(np.float32)
+    assert np.all(np.max(np.abs(q), axis=1) <= 448.0 * (1 + 2.0 ** -22))
+    arg = np.argmax(np.abs(rows), axis=1)
+    top = codes[np.arange(512), arg]
+    assert np.all((top & 0x7F) == 0x7E)
+    assert np.all(((top >> 7) & 1) == np.signbit(rows[np.arange(512), arg]))
+
+
+def test_fp8_row_exact_on_scaled_e4m3_grid():
+    """Rows of E4M3 values times 2^e whose max is 448 * 2^e have scale exactly 2^e,
+    so they quantise without error."""
+    rng = np.random.default_rng(14)
+    grid = np.concatenate([codecs.E4M3_VALUES, -codecs.E4M3_VALUES])
+    for e in range(-20, 21, 4):
+        rows = rng.choice(grid, size=(32, 128))
+        rows[np.arange(32), rng.integers(0, 128, 32)] = rng.choice([448.0, -448.0], 32)
+        rows = (rows * 2.0 ** e).astype(np.float32)
+        codes, s = codecs.fp8_row_quantize(rows)
+        np.testing.assert_array_equal(s, np.float32(2.0 ** e))
+        np.testing.assert_array_equal(codecs.fp8_row_dequantize(codes, s), rows)
