@@ -541,6 +541,19 @@ int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream)
   return ok();
 }
 
+int rssm_get_lengths(rssm_handle *h, int32_t *len_dev, int32_t *pending_dev, rssm_stream_t stream) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (!len_dev || !pending_dev) return fail(RSSM_ERR_INVALID_ARG, "len or pending is NULL");
+  const size_t n = sizeof(int32_t) * (size_t)h->d.batch;
+  cudaError_t e = cudaMemcpyAsync(len_dev, h->meta + h->lay.meta_len_off, n, cudaMemcpyDeviceToDevice,
+                                  (cudaStream_t)stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(pending_dev, h->meta + h->lay.meta_pending_off, n, cudaMemcpyDeviceToDevice,
+                        (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "copying the window lengths");
+  return ok();
+}
+
 int rssm_get_status(rssm_handle *h, uint32_t *bits, int clear, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!bits) return fail(RSSM_ERR_INVALID_ARG, "bits is NULL");

@@ -34,7 +34,7 @@ EXPORTED = [
     "rssm_get_status", "rssm_last_error_string", "rssm_launch_count",
     "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
     "rssm_branch", "rssm_restore", "rssm_get_slots",
-    "rssm_state_bytes", "rssm_export_state", "rssm_import_state",
+    "rssm_state_bytes", "rssm_export_state", "rssm_import_state", "rssm_get_lengths",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -83,6 +83,7 @@ def lib():
         L.rssm_conventional_step.argtypes = [vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_conventional_step_quantized.argtypes = [vp, vp, vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_get_bookkeeping.argtypes = [vp, vp, vp]
+        L.rssm_get_lengths.argtypes = [vp, vp, vp, vp]
         L.rssm_branch.argtypes = [vp, vp, vp]
         L.rssm_restore.argtypes = [vp, vp, vp]
         L.rssm_get_slots.argtypes = [vp, vp, vp]

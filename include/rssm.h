@@ -77,6 +77,10 @@ enum {
   RSSM_STATUS_STATE = 1u << 1,    /* row refused: drafts pending / bad rollback count  */
   RSSM_STATUS_TIMEOUT = 1u << 2   /* a bounded wait for an asynchronous copy gave up   */
 };
+/* After RSSM_STATUS_TIMEOUT the launch that set it was cut short: its outputs,
+ * the rows' pointers and any fold it was making are unspecified, and the
+ * per-sequence arrival counters in meta may be left nonzero.  Call rssm_reset
+ * (and re-initialise the checkpoint) before using the handle again. */
 
 enum { RSSM_MAMBA2 = 1, RSSM_GDN = 2, RSSM_KDA = 3 };
 enum { RSSM_F32 = 0, RSSM_BF16 = 1 };
@@ -167,28 +171,33 @@ typedef struct {
 
 typedef struct rssm_handle rssm_handle;
 
-/* Sizes (bytes) of the four caller-owned device buffers for a descriptor, and
- * the layout inside them (layout may be NULL).  ckpt = the fp32 checkpoint;
+/* (No passage: plumbing.)  Sizes (bytes) of the four caller-owned device
+ * buffers for a descriptor, and the layout inside them (layout may be NULL).  ckpt = the fp32 checkpoint;
  * read_copy is 0 for RSSM_READ_FP32.  desc.branching doubles the checkpoint
  * and read copy (2B slots) and adds the branch scratch and meta arrays. */
 int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes,
                         size_t *buf_bytes, size_t *read_copy_bytes,
                         size_t *meta_bytes, rssm_layout *layout);
 
-/* Validate the descriptor and bind the caller's device buffers to a new
- * handle (*out).  ckpt_dev holds the caller-initialised fp32 checkpoint.
+/* The layer storage [summary ¶2: a checkpoint plus a buffer of recent
+ * inputs].  Validate the descriptor and bind the caller's device buffers to a
+ * new handle (*out).  ckpt_dev holds the caller-initialised fp32 checkpoint.
  * Nothing is enqueued: the meta region must start zeroed (rssm_reset does it)
  * and the read copy must be built with rssm_quantize_read_copy before the
  * first decode when read_fmt != RSSM_READ_FP32. */
 int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev,
                 void *read_copy_dev, void *meta_dev, rssm_handle **out);
+/* (No passage: plumbing.)  Free the host handle; the caller's buffers are
+ * untouched.  NULL: RSSM_ERR_INVALID_ARG. */
 int rssm_destroy(rssm_handle *h);
 
-/* Zero the meta region (empty windows, no drafts, status clear); branching
- * layers: every sequence back to slot b. */
+/* (No passage: plumbing.)  Zero the meta region (empty windows, no drafts,
+ * status clear, arrival counters zero); branching layers: every sequence back
+ * to slot b.  Enqueued on `stream`. */
 int rssm_reset(rssm_handle *h, rssm_stream_t stream);
 
-/* Mamba-2 per-head parameters A[H] (< 0) and D[H], fp32 device arrays kept
+/* (No passage: plumbing; the parameters of the Mamba-2 recurrence above.)
+ * Mamba-2 per-head parameters A[H] (< 0) and D[H], fp32 device arrays kept
  * by pointer (they must outlive the handle).  Required before any Mamba-2
  * compute call; ignored for GDN. */
 int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev);
@@ -300,6 +309,9 @@ int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev,
  * afford cudaMalloc's implicit synchronisation.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is cached per device index for the life of the process,
+ *     which assumes one CUDA context per device (no cudaDeviceReset between
+ *     calls).
  *   - Each call clears the counters it uses (cudaMemsetAsync on `stream`).
  *   - All calls share the one array: calls that may run concurrently on the
  *     GPU (different streams, different handles) race and must not overlap.
@@ -335,14 +347,15 @@ int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream)
  */
 int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream);
 
-/* The checkpoint slot each sequence reads, after the folds of the calls
- * enqueued so far (device int32 [B]); its checkpoint is ckpt slot out[b].
+/* [guide "The State-Storage Bottleneck in Branching Workloads"]  The
+ * checkpoint slot each sequence reads, after the folds of the calls enqueued
+ * so far (device int32 [B]); its checkpoint is ckpt slot out[b].
  * RSSM_ERR_STATE if the handle was created with branching = 0. */
 int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream);
 
 /*
- * State export / import to host (serving-side preemption, migration between
- * processes or GPUs).  The blob is the layer's whole replay state in one host
+ * (No passage: plumbing for serving.)  State export / import to host
+ * (serving-side preemption, migration between processes or GPUs).  The blob is the layer's whole replay state in one host
  * buffer: checkpoint (every slot) | read copy | ring buffers | meta (pointers,
  * slots, status), in that order, raw bytes; rssm_state_bytes gives its size.
  * Import requires a handle created from the same descriptor.  Both are plain
@@ -356,20 +369,31 @@ int rssm_state_bytes(rssm_handle *h, size_t *bytes);
 int rssm_export_state(rssm_handle *h, void *host_dst, size_t bytes, rssm_stream_t stream);
 int rssm_import_state(rssm_handle *h, const void *host_src, size_t bytes, rssm_stream_t stream);
 
-/* Copy the per-sequence pointers into out_dev (device int32 [4, B]: start,
- * len, pending, flushes). */
+/* The window pointers [summary ¶3: drafts are appended and dropped by moving
+ * a pointer].  Copy the committed lengths into len_dev and the pending draft
+ * counts into pending_dev (device int32 [B] each), enqueued on `stream`
+ * (plain device-to-device copies).  NULL pointers: RSSM_ERR_INVALID_ARG. */
+int rssm_get_lengths(rssm_handle *h, int32_t *len_dev, int32_t *pending_dev,
+                     rssm_stream_t stream);
+
+/* All per-sequence pointers [summary ¶3]: copy them into out_dev (device
+ * int32 [4, B]: start, len, pending, flushes), one kernel launch. */
 int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev,
                          rssm_stream_t stream);
 
-/* Synchronise `stream` and return the sticky device status bits in *bits
- * (host pointer).  clear != 0 resets them afterwards. */
+/* (No passage: plumbing.)  Synchronise `stream` and return the sticky device
+ * status bits in *bits (host pointer).  clear != 0 resets them afterwards. */
 int rssm_get_status(rssm_handle *h, uint32_t *bits, int clear,
                     rssm_stream_t stream);
 
-/* Thread-local text describing the last error on this thread ("" if none). */
+/* (No passage: plumbing.)  Thread-local text describing the last error on
+ * this thread ("" if none). */
 const char *rssm_last_error_string(void);
 
-/* Number of GPU kernels this library has launched in this process. */
+/* (No passage: plumbing.)  Number of GPU kernels this library has launched
+ * in this process.  Kernel launches only: the memsets and copies some calls
+ * enqueue (rssm_reset, rssm_get_status, the static-scratch clear, state
+ * export/import, rssm_get_lengths) are not counted. */
 uint64_t rssm_launch_count(void);
 
 #ifdef __cplusplus

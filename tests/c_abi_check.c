@@ -40,6 +40,7 @@ int main(void) {
   if (rssm_decode_step(NULL, NULL, NULL, NULL) != RSSM_ERR_INVALID_ARG) return 8;
   size_t n = 0;
   if (rssm_state_bytes(NULL, &n) != RSSM_ERR_INVALID_ARG) return 9;
+  if (rssm_get_lengths(NULL, NULL, NULL, NULL) != RSSM_ERR_INVALID_ARG) return 10;
   printf("c abi ok\n");
   return 0;
 }

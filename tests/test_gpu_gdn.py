@@ -102,27 +102,6 @@ def test_window_one_equals_conventional_update():
         assert rel_err(layer.ckpt.cpu(), state.cpu()) < 2e-6
 
 
-def test_serving_batch_sampled_rows():
-    """Batch 256, 32 heads, d_k = d_v = 128, bf16 q/k/v, L = 16, 1024 steps, in the
-    launch configuration the bench times; sampled sequences checked every step."""
-    shape = si.GDN_SERVING
-    rows = [7, 200]
-    layer, S0 = gdn_layer(shape)
-    S = S0[rows].double().numpy()
-    out = torch.empty(256, 32, 128, device=DEV)
-    worst = 0.0
-    for t in range(1024):
-        tok = si.gdn_tokens(shape, t)
-        layer.decode_step(dev_inputs(tok, GDN_KEYS), out)
-        S, o = _oracle_step(S, {k: v[rows] for k, v in tok.items()})
-        worst = max(worst, assert_close(out[rows].cpu(), o, TOL["bf16"], f"step {t}"))
-    layer.flush()
-    assert_close(layer.ckpt[rows].cpu(), S, TOL["bf16"], "checkpoint")
-    bk = layer.get_bookkeeping().cpu()
-    assert torch.all(bk[1] == 0) and torch.all(bk[3] == 64)
-    print(f"max scaled error over 1024 steps {worst:.2e}")
-
-
 @pytest.mark.parametrize("k,L", [(1, 8), (3, 8), (4, 8), (1, 1)])
 def test_verify_rollback(k, L):
     """Verify rounds with seeded acceptance and decode steps in between; with

@@ -54,29 +54,6 @@ def test_decode_and_folds_against_oracle(L, dtype):
     assert layer.get_status() == 0
 
 
-def test_serving_batch_sampled_rows():
-    """Batch 256, 32 heads, d_k = d_v = 128, bf16 q/k/v, L = 16, in the launch
-    configuration the bench times; sampled sequences checked every step through
-    ten folds."""
-    shape = si.KDA_SERVING
-    rows = [7, 200]
-    layer, S0 = kda_layer(shape)
-    S = to64(S0[rows])
-    out = torch.empty(256, 32, 128, device=DEV)
-    worst = 0.0
-    for t in range(160):
-        tok = si.kda_tokens(shape, t)
-        layer.decode_step(dev_inputs(tok, KDA_KEYS), out)
-        S, y = _step(S, tok64({k: v[rows] for k, v in tok.items()}))
-        worst = max(worst, assert_close(out[rows].cpu(), y, TOL["bf16"], f"step {t}"))
-    layer.flush()   # 160 tokens = 10 full windows: the checkpoint is the state
-    assert_close(layer.ckpt[rows].cpu(), S, TOL["bf16"], "checkpoint")
-    bk = layer.get_bookkeeping().cpu()
-    assert torch.all(bk[1] == 0) and torch.all(bk[3] == 10)
-    assert layer.get_status() == 0
-    print(f"max scaled error over 160 steps {worst:.2e}")
-
-
 def test_conventional_kernel_against_oracle():
     shape = si.KDALayer(batch=4, nheads=8, dk=128, dv=128, window=16, dtype="bf16", state_std=0.05)
     layer, S0 = kda_layer(shape)

@@ -107,28 +107,6 @@ def test_window_one_equals_conventional_update():
         assert rel_err(layer.ckpt.cpu(), state.cpu()) < 1e-6
 
 
-def test_serving_batch_sampled_rows():
-    """Batch 256, 128 heads, P=64, N=128, G=8, bf16 inputs, L=16, 1024 steps, in the
-    launch configuration the bench times; sampled sequences checked every step."""
-    shape = si.MAMBA2_SERVING
-    rows = [5, 254]
-    layer, A, D, h0 = m2_layer(shape)
-    h = h0[rows].double().numpy()
-    out = torch.empty(shape.batch, shape.nheads, shape.headdim, device=DEV)
-    worst = 0.0
-    for t in range(1024):
-        tok = si.mamba2_tokens(shape, t)
-        layer.decode_step(dev_inputs(tok, M2_KEYS), out)
-        sub = {k: v[rows] for k, v in tok.items()}
-        h, y = _oracle_step(h, sub, A, D)
-        worst = max(worst, assert_close(out[rows].cpu(), y, TOL["bf16"], f"step {t}"))
-    layer.flush()
-    assert_close(layer.ckpt[rows].cpu(), h, TOL["bf16"], "checkpoint")
-    bk = layer.get_bookkeeping().cpu()
-    assert torch.all(bk[1] == 0) and torch.all(bk[3] == 64)
-    print(f"max scaled error over 1024 steps {worst:.2e}")
-
-
 @pytest.mark.parametrize("k", [1, 3, 4])
 def test_verify_rollback(k):
     """Rounds of verify(k) + rollback with seeded acceptance, decode steps in

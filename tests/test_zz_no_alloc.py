@@ -5,8 +5,12 @@ library extra device memory when they decode: code recording decode steps
 into a CUDA graph (nothing may be allocated inside a capture), serving
 engines that reserve all device memory when they start, and tight loops that
 cannot pay for cudaMalloc's implicit synchronisation.  It keeps the replay
-kernel's per-sequence arrival counters in an array inside the library.  Its
-results must be those of the ordinary decode step, call after call.
+kernel's per-sequence arrival counters in an array inside the library.  It
+runs the same kernel on the same inputs as the ordinary decode step, so its
+outputs, ring pointers and checkpoint must be bit-identical to that call's,
+call after call, for every layer type (the counters expect a different number
+of arrivals per sequence in each: groups x head chunks for Mamba-2, head chunks
+for Gated DeltaNet, heads for KDA).
 
 This file is collected last on purpose (its name sorts after the others), so
 a run that stops at the first failure has run every other test first.
@@ -17,7 +21,7 @@ import pytest
 import torch
 
 import seeded_inputs as si
-from gpu_common import DEV, M2_KEYS, assert_close, dev_inputs, m2_layer
+from gpu_common import DEV, GDN_KEYS, KDA_KEYS, M2_KEYS, dev_inputs, gdn_layer, kda_layer, m2_layer
 from hybrid_ssm_decode_replayssm_b200 import rssm
 
 pytestmark = pytest.mark.gpu
@@ -29,24 +33,40 @@ def _static_scratch_decode(layer, inputs, out):
         layer.handle, arr, out.data_ptr(), torch.cuda.current_stream().cuda_stream))
 
 
-def test_static_scratch_decode_matches_decode_step():
-    # 64 sequences x 4 groups = 256 items: more items than resident CTAs, so every
-    # CTA works through several items and 4 CTAs meet on each sequence's counter.
-    # Window 2: the second call fills the window and folds it into the checkpoint.
-    shape = si.Mamba2Layer(batch=64, nheads=16, headdim=64, dstate=128, ngroups=4, window=2,
-                           dtype="bf16", state_std=0.1, max_draft=2)
-    ref, _, _, _ = m2_layer(shape, seed=3)
-    nal, _, _, _ = m2_layer(shape, seed=3)
-    y_ref = torch.empty(64, 16, 64, device=DEV)
+def _pair(kind):
+    """Two identical layers (same seeds), their token function, keys and output shape.
+    Window 2: the second call fills the window and folds it into the checkpoint."""
+    if kind == "mamba2":
+        # 64 sequences x 4 groups = 256 items: more items than resident CTAs, so every
+        # CTA works through several items and 4 CTAs meet on each sequence's counter.
+        shape = si.Mamba2Layer(batch=64, nheads=16, headdim=64, dstate=128, ngroups=4, window=2,
+                               dtype="bf16", state_std=0.1, max_draft=2)
+        make = lambda: m2_layer(shape, seed=3)[0]
+        return make(), make(), (lambda t: si.mamba2_tokens(shape, t, seed=3)), M2_KEYS, (64, 16, 64)
+    if kind == "gdn":
+        shape = si.GDNLayer(batch=64, nheads=8, dk=128, dv=128, window=2, dtype="bf16", state_std=0.05,
+                            max_draft=2)
+        make = lambda: gdn_layer(shape, seed=3)[0]
+        return make(), make(), (lambda t: si.gdn_tokens(shape, t, seed=3)), GDN_KEYS, (64, 8, 128)
+    shape = si.KDALayer(batch=16, nheads=8, dk=128, dv=128, window=2, dtype="bf16", state_std=0.05)
+    make = lambda: kda_layer(shape, seed=3)[0]
+    return make(), make(), (lambda t: si.kda_tokens(shape, t, seed=3)), KDA_KEYS, (16, 8, 128)
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_static_scratch_decode_matches_decode_step(kind):
+    ref, nal, tokens, keys, out_shape = _pair(kind)
+    y_ref = torch.empty(out_shape, device=DEV)
     y_nal = torch.full_like(y_ref, float("nan"))
     for t in range(2):                       # two calls in a row
-        ins = dev_inputs(si.mamba2_tokens(shape, t, seed=3), M2_KEYS)
+        ins = dev_inputs(tokens(t), keys)
         ref.decode_step(ins, y_ref)
         _static_scratch_decode(nal, ins, y_nal)
         torch.cuda.synchronize()
-        assert_close(y_nal.cpu(), y_ref.cpu(), 2e-3, f"call {t}: outputs")
+        assert torch.equal(y_nal, y_ref), f"call {t}: outputs differ"
         assert torch.equal(nal.get_bookkeeping(), ref.get_bookkeeping()), f"call {t}: ring pointers"
-    assert_close(nal.ckpt.cpu(), ref.ckpt.cpu(), 2e-3, "checkpoint after the fold")
+    assert torch.equal(nal.ckpt, ref.ckpt), "checkpoint after the fold"
+    assert int(ref.get_bookkeeping()[3].min()) == 1, "the second call must fold every sequence"
     assert nal.get_status() == 0 and ref.get_status() == 0
 
 
