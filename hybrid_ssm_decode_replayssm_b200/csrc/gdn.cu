@@ -35,6 +35,7 @@
 // unit each warp owns 8 state rows; a row is spread over 8 lanes (4 chunks of
 // 4 columns each), so its dot products reduce in three shuffle steps.
 #include "rssm_device.cuh"
+#include "umma.cuh"
 
 namespace rssm {
 namespace {
@@ -83,9 +84,20 @@ __device__ __forceinline__ void scale4(float4 &t, float c) { t.x *= c; t.y *= c;
 // betas of the item's heads, fp32 k/q/v of the new tokens, the committed
 // window k rows of the item's heads (input dtype), per-head output scalars,
 // fold scalars, per-warp scratch.
+// Folds of layers that read the fp32 checkpoint with bf16 inputs run on the
+// tensor cores (tcgen05): the rank-l update of a unit, D^T[c][r] =
+// sum_i k_i[c] (fw_i w_i[r]), is one M = 128 (key columns) x N = 64 (value
+// rows) x K = l bf16 MMA chain per unit with an fp32 accumulator in TMEM.  The
+// k rows are bf16 already (exact); each weighted w value is split into three
+// bf16 parts (hi, mid, lo; their sum is the fp32 value to 2^-24), so the
+// products are exact and only the fp32 accumulation rounds, as on the CUDA
+// cores.  The epilogue adds e^{G} S from the stage and stores.
+template <typename Tin, int RF>
+constexpr bool umma_fold() { return RF == RSSM_READ_FP32 && sizeof(Tin) == 2; }
+
 struct Layout {
   int woff, voff, stage_bytes;
-  int sg, sbeta, kqv, kbuf, hso, fold, warp, warp_floats, group_floats;
+  int sg, sbeta, kqv, kbuf, hso, fold, warp, warp_floats, umma, umma_kg, group_floats;
 };
 template <typename Tin, int RF, int MAXM>
 __host__ __device__ inline Layout make_layout(int L, int hc) {
@@ -107,7 +119,13 @@ __host__ __device__ inline Layout make_layout(int L, int hc) {
   y.warp = (y.fold + fold_floats + 3) & ~3;
   // per warp: red[8][MAXM][2] | win[8][MAXM][2] | wnew[MAXM][8] | U[L][8] (re-solving layers)
   y.warp_floats = (5 * MAXM * RPW + (kResolve ? L * RPW : 0) + 3) & ~3;
-  y.group_floats = (y.warp + kGroupWarps * y.warp_floats + 31) & ~31;
+  // tensor-core fold operands (MN-major bf16 tiles, 128-byte aligned): A = the
+  // window's k rows [DK columns x 16 nk entries], B = three parts of the
+  // weighted w [HALF rows x 16 nk entries]; nk = ceil(L / 16) MMA K-steps
+  y.umma_kg = 2 * ((L + 15) / 16);
+  y.umma = (y.warp + kGroupWarps * y.warp_floats + 31) & ~31;
+  const int umma_floats = umma_fold<Tin, RF>() ? (DK / 8 + 3 * HALF / 8) * y.umma_kg * 128 / 4 : 0;
+  y.group_floats = (y.umma + umma_floats + 31) & ~31;
   return y;
 }
 
@@ -159,8 +177,12 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   constexpr int RB = rc_row_bytes<RF>();
   constexpr int SR = rc_scale_row_bytes<RF>();
   constexpr int HSO = MAXM + 2 * MAXM * kMaxW;   // per head: dec[MAXM] | Mk[MAXM][32] | Mq[MAXM][32]
+  constexpr bool kUmma = umma_fold<Tin, RF>();
+  constexpr uint32_t kTmemCols = 2 * HALF;        // one 64-column fp32 accumulator per consumer group
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
+  __shared__ uint64_t mma_bar[kGroups];           // tensor-core fold completion, one per group
+  __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -185,10 +207,19 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kGroupWarps);
     }
+    for (int g = 0; g < kGroups; ++g) mbar_init(&mma_bar[g], 1);
     abort_flag = 0;
     mbar_fence_init();
   }
+  if constexpr (kUmma) {
+    if (warp == 0) {   // TMEM for both groups' fold accumulators; freed by warp 0 at the end
+      umma::alloc(&tmem_base, kTmemCols);
+      umma::relinquish();
+    }
+    umma::fence_before_sync();
+  }
   __syncthreads();
+  if constexpr (kUmma) umma::fence_after_sync();
 
   auto item_of = [&](int k, int &b, int &chunk) {
     const int item = (int)blockIdx.x + k * (int)gridDim.x;
@@ -224,7 +255,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         if (u_ == 0 || mbar_try_wait(&empty[s_], (uint32_t)((u_ - 1) & 1))) g = c;
       }
       if (g < 0) {
-        if (*abort || clock64() - idle_since > 2000000000LL) {
+        if (*abort || clock64() - idle_since > a.wait_limit) {
           timed_out = true;
           break;
         }
@@ -473,7 +504,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       s = base + t % Rg;
       use = t / Rg;
     };
-    auto wait_stage = [&]() -> bool { return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort); };
+    auto wait_stage = [&]() -> bool { return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit); };
     auto release_stage = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -485,6 +516,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     // the warp skips its work but passes every group barrier, whose OR
     // reduction spreads the failure, so all warps keep the same barrier sequence.
     bool failed = false;
+    int mma_uses = 0;   // completed tensor-core folds of this group (parity of mma_bar[gi])
     for (int jh = 0; jh < hc; ++jh) {
       const int h = h0 + jh;
       const size_t bh = bh0 + jh;
@@ -519,6 +551,8 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         if (hf == 0 && (pre || post) && named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
         const bool have = !failed && wait_stage();
         if (!have) failed = true;
+        // a tensor-core fold has group barriers inside: every warp must agree on doing it
+        if (kUmma && hf == 1 && (pre || post) && named_sync_or(bar_id, kGroupThreads, failed)) failed = true;
         bool released = false;
         const uint8_t *sb = smem + s * Y.stage_bytes;
         const float *wst = reinterpret_cast<const float *>(sb + Y.woff);   // cached w, committed entries
@@ -699,8 +733,103 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           if constexpr (kResolve) __syncwarp();   // U is reused by the next fold
         };
 
+        // ---- tensor-core fold of the unit's 64 rows by the whole group: x <- decF x +
+        //      sum_i fw_i w_i[row] k_i^T over the window [i0, i0 + nf), as D^T[c][r] =
+        //      sum_i k_i[c] (fw_i w_i[r]) (M = 128 key columns, N = 64 rows, K = the
+        //      entries, zero padded to 16 per MMA step).  Operands: A = the k rows
+        //      (bf16, exact), B = three bf16 parts of fw_i w_i[r], each warp writing its
+        //      own 8 rows.  The epilogue thread of key column c adds decF S[r][c] from
+        //      the stage for 32 rows r and stores the result to the stage (to_stage:
+        //      a pre-fold whose result the outputs read) and/or to the checkpoint.
+        auto fold_tc = [&](int i0, int nf, int which, bool to_stage, bool to_global) {
+          const float *fwv = fw + which * (kMaxW + 1);
+          const int KG = Y.umma_kg, KE = KG * 8;
+          uint8_t *uA = reinterpret_cast<uint8_t *>(G + Y.umma);
+          uint8_t *uB = uA + (DK / 8) * KG * 128;
+          const int partB = (HALF / 8) * KG * 128;
+          for (int idx = gt; idx < KE * (DK / 8); idx += kGroupThreads) {
+            const int i = idx / (DK / 8), cc = idx - i * (DK / 8);
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (i < nf) {
+              const int e = i0 + i;
+              if (e < n) {
+                val = *reinterpret_cast<const uint4 *>(kb + (size_t)e * DK + 8 * cc);
+              } else {   // a new token's k (bf16 values widened exactly): back to bf16
+                const float4 lo4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc);
+                const float4 hi4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc + 4);
+                const __nv_bfloat162 p0 = __floats2bfloat162_rn(lo4.x, lo4.y), p1 = __floats2bfloat162_rn(lo4.z, lo4.w);
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(hi4.x, hi4.y), p3 = __floats2bfloat162_rn(hi4.z, hi4.w);
+                val = make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
+                                 *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
+              }
+            }
+            *reinterpret_cast<uint4 *>(uA + umma::mn_offset(8 * cc, i, KG)) = val;
+          }
+          for (int p = lane; p < KE * RPW; p += 32) {
+            const int i = p >> 3, r8 = p & 7;
+            float x = 0.0f;
+            if (i < nf) {
+              const int e = i0 + i;
+              x = fwv[i] * (e < n ? wst[e * HALF + urow0 + r8] : wnew[(e - n) * RPW + r8]);
+            }
+            uint16_t xh, xm, xl;
+            umma::split3_bf16(x, xh, xm, xl);
+            const uint32_t off = umma::mn_offset(urow0 + r8, i, KG);
+            *reinterpret_cast<uint16_t *>(uB + off) = xh;
+            *reinterpret_cast<uint16_t *>(uB + partB + off) = xm;
+            *reinterpret_cast<uint16_t *>(uB + 2 * partB + off) = xl;
+          }
+          fence_proxy_async();   // operands written by this thread -> visible to the tensor core
+          umma::fence_before_sync();
+          named_sync(bar_id, kGroupThreads);
+          const uint32_t tm = tmem_base + (uint32_t)(gi * HALF);
+          if (gt == 0) {
+            umma::fence_after_sync();
+            constexpr uint32_t idesc = umma::idesc_bf16_f32_mn(DK, HALF);
+            for (int part = 0; part < 3; ++part)
+              for (int ks = 0; ks < KG / 2; ++ks)
+                umma::mma_bf16(tm, umma::smem_desc_mn(smem_u32(uA) + 256 * ks, 128, KG * 128),
+                               umma::smem_desc_mn(smem_u32(uB + part * partB) + 256 * ks, 128, KG * 128), idesc,
+                               part > 0 || ks > 0);
+            umma::commit(&mma_bar[gi]);
+          }
+          // the MMAs always complete: wait without the abort flag (bounded), so
+          // that TMEM is never released under a running MMA
+          const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
+          ++mma_uses;
+          umma::fence_after_sync();
+          if (!ok) {
+            *abort = 1;
+            failed = true;
+            return;
+          }
+          const int q = gw & 3, c = 32 * q + lane, rh = (gw >> 2) * 32;
+          float d[32];
+          umma::ld_32x32b_x32(tm + ((uint32_t)(32 * q) << 16) + (uint32_t)rh, d);
+          umma::fence_before_sync();
+          const float dF = decF[which];
+          float *tile = reinterpret_cast<float *>(const_cast<uint8_t *>(sb));
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int r = rh + j;
+            const float val = fmaf(dF, tile[r * DK + c], d[j]);
+            if (to_stage) tile[r * DK + c] = val;
+            if (to_global) __stcs(hc_rows + (size_t)r * DK + c, val);
+          }
+        };
+
         // ---- the read view of this warp's rows, after a pre-fold if one is due
         float4 v[2][4];   // read view (re-solving layers); fp32 layers read f
+        if constexpr (kUmma) {
+          if (pre) {   // the new tokens do not fit: fold the committed window first, into the stage
+            fold_tc(0, nf0, 0, true, !post);
+            if (named_sync_or(bar_id, kGroupThreads, failed)) failed = true;   // the folded tile is complete
+            if (failed) {
+              if (have) release_stage();
+              continue;
+            }
+          }
+        }
         if constexpr (!kResolve) {
           const float *tile = reinterpret_cast<const float *>(sb);
 #pragma unroll
@@ -709,7 +838,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             for (int c = 0; c < 4; ++c)
               f[r][c] = *reinterpret_cast<const float4 *>(tile + (size_t)(r == 0 ? row_a : row_b) * DK + 32 * c + 4 * j8);
         }
-        if (pre) {   // the new tokens do not fit: fold the committed window first
+        if (!kUmma && pre) {   // the new tokens do not fit: fold the committed window first
           fold(f, 0, nf0, 0);
 #pragma unroll
           for (int r = 0; r < 2; ++r)
@@ -831,7 +960,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
           __syncwarp();
         }
 
-        if (post) {   // the decode filled the window: fold all of it
+        if (kUmma && post) {   // the decode filled the window: fold all of it (tensor cores)
+          fold_tc(w0, nf1, 1, false, true);
+        } else if (post) {   // the decode filled the window: fold all of it
           fold(f, w0, nf1, 1);
 #pragma unroll
           for (int r = 0; r < 2; ++r)
@@ -847,7 +978,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     const bool any_abort = named_sync_or(bar_id, kGroupThreads, failed || *abort != 0);
     if (any_abort) {
       if (gt == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
-      return;
+      break;   // every consumer thread still meets the others at the TMEM release below
     }
     if (!rp.refuse && gt == 0) {
       __threadfence();
@@ -873,6 +1004,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         a.len[b] = n2;
         a.flushes[b] = fl;
       }
+    }
+  }
+  if constexpr (kUmma) {   // both groups are done with their accumulators
+    umma::fence_before_sync();
+    named_sync(3, kConsumers);
+    if (warp == 0) {
+      umma::fence_after_sync();
+      umma::dealloc(tmem_base, kTmemCols);
     }
   }
 }

@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     int b_e = 0, g_e = 0, chunk_e = 0;
     int issued = 0;
     for (int seq = 0; seq < total_seq; ++seq) {
-      if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort)) {
+      if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort, a.wait_limit)) {
         atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
         break;
       }
@@ -481,14 +481,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     const int seq_base = (k >> 1) * 2 * hc;
     int s = seq_base % stages, use = seq_base / stages;
     bool inter = false;
-    if (wait_flag_at_least(&stage_use[s], use, abort)) {   // the pair's first head is issued
+    if (wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit)) {   // the pair's first head is issued
       __threadfence_block();
       inter = *reinterpret_cast<volatile int *>(&pair_inter[(k >> 1) % kPairSlots]) != 0;
     }
     // wait until the producer has requested use `use` of stage s, then for the data
     auto wait_stage = [&]() -> bool {
-      if (!wait_flag_at_least(&stage_use[s], use, abort)) return false;
-      return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort);
+      if (!wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit)) return false;
+      return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit);
     };
     constexpr int hstep = kMma ? 2 : 1;   // heads taken by this warp: sub, sub + hstep, ...
     {

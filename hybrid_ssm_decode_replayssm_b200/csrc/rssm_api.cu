@@ -16,6 +16,7 @@ struct rssm_handle {
   float *ckpt;
   uint8_t *buf, *rc, *meta;
   const float *A, *D;
+  long long wait_limit;
 };
 
 namespace {
@@ -148,6 +149,7 @@ rssm::StepArgs step_args(const rssm_handle *h, int mode, int m) {
   a.L = d.window; a.cap = (int)h->lay.cap;
   a.m = m; a.mode = mode; a.auto_flush = d.auto_flush != 0;
   a.out_scale = d.out_scale;
+  a.wait_limit = h->wait_limit;
   a.A = h->A; a.D = h->D;
   a.hc = h->ckpt;
   if (d.branching) {
@@ -261,6 +263,7 @@ int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev, void
   h->buf = static_cast<uint8_t *>(buf_dev);
   h->rc = desc->read_fmt == RSSM_READ_FP32 ? nullptr : static_cast<uint8_t *>(read_copy_dev);
   h->meta = static_cast<uint8_t *>(meta_dev);
+  h->wait_limit = rssm::kDefaultWaitLimit;
   *out = h;
   return ok();
 }
@@ -289,6 +292,13 @@ int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev) {
     return fail(RSSM_ERR_INVALID_ARG, "A and D must not be NULL");
   h->A = A_dev;
   h->D = D_dev;
+  return ok();
+}
+
+int rssm_set_wait_limit(rssm_handle *h, long long cycles) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (cycles < 0) return fail(RSSM_ERR_INVALID_ARG, "wait limit must be >= 0 (0 = default)");
+  h->wait_limit = cycles == 0 ? rssm::kDefaultWaitLimit : cycles;
   return ok();
 }
 

@@ -43,7 +43,12 @@ struct StepArgs {
   // bookkeeping
   int32_t *start, *len, *pending, *flushes, *arrivals;
   uint32_t *status;
+  // give-up limit (SM clock cycles) of the bounded waits on copies and on the
+  // other warps; waits for the tensor cores and the final drain keep their own
+  long long wait_limit;
 };
+
+constexpr long long kDefaultWaitLimit = 2000000000LL;   // about a second at B200 clocks
 
 struct ConvArgs {
   int B, H, G, hpg, R, C;

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(HERE, "librssm.so")
 
 RSSM_OK, RSSM_ERR_INVALID_ARG, RSSM_ERR_UNSUPPORTED = 0, 1, 2
 RSSM_ERR_CAPACITY, RSSM_ERR_STATE, RSSM_ERR_CUDA, RSSM_ERR_TIMEOUT = 3, 4, 5, 6
-RSSM_STATUS_CAPACITY, RSSM_STATUS_STATE = 1, 2
+RSSM_STATUS_CAPACITY, RSSM_STATUS_STATE, RSSM_STATUS_TIMEOUT = 1, 2, 4
 RSSM_MAMBA2, RSSM_GDN, RSSM_KDA = 1, 2, 3
 RSSM_F32, RSSM_BF16 = 0, 1
 RSSM_READ_FP32, RSSM_READ_FP8_E4M3_ROW, RSSM_READ_NVFP4 = 0, 1, 2
@@ -35,6 +35,7 @@ EXPORTED = [
     "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
     "rssm_branch", "rssm_restore", "rssm_get_slots",
     "rssm_state_bytes", "rssm_export_state", "rssm_import_state", "rssm_get_lengths",
+    "rssm_set_wait_limit",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -84,6 +85,7 @@ def lib():
         L.rssm_conventional_step_quantized.argtypes = [vp, vp, vp, vp, vp, C.POINTER(vp), vp, vp]
         L.rssm_get_bookkeeping.argtypes = [vp, vp, vp]
         L.rssm_get_lengths.argtypes = [vp, vp, vp, vp]
+        L.rssm_set_wait_limit.argtypes = [vp, C.c_longlong]
         L.rssm_branch.argtypes = [vp, vp, vp]
         L.rssm_restore.argtypes = [vp, vp, vp]
         L.rssm_get_slots.argtypes = [vp, vp, vp]

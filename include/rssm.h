@@ -188,7 +188,7 @@ int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes,
 int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev,
                 void *read_copy_dev, void *meta_dev, rssm_handle **out);
 /* (No passage: plumbing.)  Free the host handle; the caller's buffers are
- * untouched.  NULL: RSSM_ERR_INVALID_ARG. */
+ * untouched.  NULL is accepted and does nothing. */
 int rssm_destroy(rssm_handle *h);
 
 /* (No passage: plumbing.)  Zero the meta region (empty windows, no drafts,
@@ -201,6 +201,14 @@ int rssm_reset(rssm_handle *h, rssm_stream_t stream);
  * by pointer (they must outlive the handle).  Required before any Mamba-2
  * compute call; ignored for GDN. */
 int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev);
+
+/* (No passage: plumbing.)  Give-up limit, in SM clock cycles, of the replay
+ * kernels' bounded waits (for a stage's asynchronous copies, for the other
+ * warps to release a stage).  A wait that runs out sets RSSM_STATUS_TIMEOUT
+ * and the launch stops early, with the device context intact (see above).
+ * 0 restores the default (2e9 cycles, about a second); negative values:
+ * RSSM_ERR_INVALID_ARG.  Applies to the calls enqueued after it. */
+int rssm_set_wait_limit(rssm_handle *h, long long cycles);
 
 /*
  * Decode one token per sequence [summary ¶2-3]: append its inputs to the
