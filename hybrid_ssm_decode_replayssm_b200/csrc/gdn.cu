@@ -119,10 +119,10 @@ __host__ __device__ inline Layout make_layout(int L, int hc) {
   y.warp = (y.fold + fold_floats + 3) & ~3;
   // per warp: red[8][MAXM][2] | win[8][MAXM][2] | wnew[MAXM][8] | U[L][8] (re-solving layers)
   y.warp_floats = (5 * MAXM * RPW + (kResolve ? L * RPW : 0) + 3) & ~3;
-  // tensor-core fold operands (MN-major bf16 tiles, 128-byte aligned): A = the
-  // window's k rows [DK columns x 16 nk entries], B = three parts of the
-  // weighted w [HALF rows x 16 nk entries]; nk = ceil(L / 16) MMA K-steps
-  y.umma_kg = 2 * ((L + 15) / 16);
+  // tensor-core fold operands (MN-major bf16 tiles, 128-byte aligned) for one
+  // block of 16 window entries: A = their k rows [DK columns x 16], B = three
+  // parts of the weighted w [HALF rows x 16]; longer windows go block by block
+  y.umma_kg = 2;
   y.umma = (y.warp + kGroupWarps * y.warp_floats + 31) & ~31;
   const int umma_floats = umma_fold<Tin, RF>() ? (DK / 8 + 3 * HALF / 8) * y.umma_kg * 128 / 4 : 0;
   y.group_floats = (y.umma + umma_floats + 31) & ~31;
@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   __shared__ uint64_t mma_bar[kGroups];           // tensor-core fold completion, one per group
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int never_set;                       // the timeout self-test waits for it
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L, cap = a.cap, m = a.m, WMAX = L + MAXM;
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     }
     for (int g = 0; g < kGroups; ++g) mbar_init(&mma_bar[g], 1);
     abort_flag = 0;
+    never_set = 0;
     mbar_fence_init();
   }
   if constexpr (kUmma) {
@@ -357,6 +359,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   const int g8 = lane >> 3, j8 = lane & 7;   // state mapping: rows g8, g8 + 4 of the warp; lane j8 of the row
   const int urow0 = gw * RPW;           // first row of this warp inside a unit
   const int row_a = urow0 + g8, row_b = urow0 + g8 + 4;
+  if (a.stall_test && blockIdx.x == 0) {   // the timeout self-test: this CTA's waits run out
+    stall_on_unset_flag(&never_set, abort, a.wait_limit);
+    if (gt == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
+  }
+
 
   for (int k = gi; k < my_items; k += kGroups) {
     int b, chunk;
@@ -382,55 +389,74 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         cp_async16(reinterpret_cast<uint8_t *>(kbuf + ((size_t)jh * L + i) * DK) + 16 * c,
                    reinterpret_cast<const uint8_t *>(kring + ((bh0 + jh) * cap + slot) * DK) + 16 * c);
       }
-      // ---- gates and betas of the item's heads; ring appends of the new gates
+      // ---- gates and betas of the item's heads (committed from the ring, new
+      //      from the inputs: raw alpha, its log is taken below), also in flight
       for (int idx = gt; idx < hc * ntot; idx += kGroupThreads) {
         const int jh = idx / ntot, i = idx - jh * ntot;
         const size_t bh = bh0 + jh;
-        float g, be;
+        const float *gsrc, *bsrc;
         if (i < n) {
-          const int slot = (st + i) % cap;
-          g = gring[bh * cap + slot];
-          be = bring[bh * cap + slot];
+          const size_t o = bh * cap + (st + i) % cap;
+          gsrc = gring + o;
+          bsrc = bring + o;
         } else {
           const size_t tok = ((size_t)b * m + (i - n)) * a.H + h0 + jh;
-          const int slot = (slot_n + (i - n)) % cap;
-          g = logf(alin[tok]);
-          be = bein[tok];
-          gring[bh * cap + slot] = g;
-          bring[bh * cap + slot] = be;
+          gsrc = alin + tok;
+          bsrc = bein + tok;
         }
-        sg[jh * WMAX + i] = g;
-        sbeta[jh * WMAX + i] = be;
+        cp_async4(sg + jh * WMAX + i, gsrc);
+        cp_async4(sbeta + jh * WMAX + i, bsrc);
       }
-      // ---- new tokens: k, q, v rows to fp32 in shared memory; k and v appended to the ring
+      // ---- new tokens: k, q, v rows to fp32 in shared memory; k and v appended
+      //      to the ring.  A thread's 16-byte loads (up to kBatch) are issued before any is used.
       constexpr int kPer = 16 / sizeof(Tin);
       constexpr int kLoads = DK / kPer;   // 16-byte loads per row
-      for (int idx = gt; idx < hc * m * 3 * kLoads; idx += kGroupThreads) {
-        const int c = (idx % kLoads) * kPer;
-        int r = idx / kLoads;
-        const int which = r % 3;   // 0 k, 1 q, 2 v
-        r /= 3;
-        const int j = r % m, jh = r / m;
-        const size_t tok = ((size_t)b * m + j) * a.H + h0 + jh;
-        const Tin *src = (which == 0 ? kin : which == 1 ? qin : vin) + tok * DK + c;
-        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src));
-        const Tin *e = reinterpret_cast<const Tin *>(&raw);
-        float *dst = kqv + ((size_t)(jh * 3 + which) * MAXM + j) * DK + c;
+      const int ntok = hc * m * 3 * kLoads;
+      constexpr int kBatch = MAXM == 1 ? 1 : 4;
+      for (int base = 0; base < ntok; base += kBatch * kGroupThreads) {
+        uint4 raw[kBatch];
 #pragma unroll
-        for (int q = 0; q < kPer; q += 4)
-          *reinterpret_cast<float4 *>(dst + q) =
-              make_float4(to_f32<Tin>(e[q]), to_f32<Tin>(e[q + 1]), to_f32<Tin>(e[q + 2]), to_f32<Tin>(e[q + 3]));
-        const size_t bh = bh0 + jh;
-        const int slot = (slot_n + j) % cap;
-        if (which == 0) {
-          *reinterpret_cast<uint4 *>(kring + (bh * cap + slot) * DK + c) = raw;
-        } else if (which == 2) {
-          const int hf = c / HALF;
-          *reinterpret_cast<uint4 *>(vring + ((bh * 2 + hf) * cap + slot) * HALF + (c - hf * HALF)) = raw;
+        for (int q = 0; q < kBatch; ++q) {
+          const int idx = base + q * kGroupThreads + gt;
+          if (idx < ntok) {
+            const int c = (idx % kLoads) * kPer, r = idx / kLoads, which = r % 3, j = (r / 3) % m, jh = r / 3 / m;
+            const size_t tok = ((size_t)b * m + j) * a.H + h0 + jh;
+            raw[q] = __ldg(reinterpret_cast<const uint4 *>((which == 0 ? kin : which == 1 ? qin : vin) + tok * DK + c));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int idx = base + q * kGroupThreads + gt;
+          if (idx >= ntok) continue;
+          const int c = (idx % kLoads) * kPer, r = idx / kLoads, which = r % 3, j = (r / 3) % m, jh = r / 3 / m;
+          const Tin *e = reinterpret_cast<const Tin *>(&raw[q]);
+          float *dst = kqv + ((size_t)(jh * 3 + which) * MAXM + j) * DK + c;
+#pragma unroll
+          for (int u = 0; u < kPer; u += 4)
+            *reinterpret_cast<float4 *>(dst + u) =
+                make_float4(to_f32<Tin>(e[u]), to_f32<Tin>(e[u + 1]), to_f32<Tin>(e[u + 2]), to_f32<Tin>(e[u + 3]));
+          const size_t bh = bh0 + jh;
+          const int slot = (slot_n + j) % cap;
+          if (which == 0) {
+            *reinterpret_cast<uint4 *>(kring + (bh * cap + slot) * DK + c) = raw[q];
+          } else if (which == 2) {
+            const int hf = c / HALF;
+            *reinterpret_cast<uint4 *>(vring + ((bh * 2 + hf) * cap + slot) * HALF + (c - hf * HALF)) = raw[q];
+          }
         }
       }
       cp_async_wait_all();
       named_sync(bar_id, kGroupThreads);
+      // ---- the new gates: ln alpha, appended with the betas to the ring (read
+      //      by the decays after the next group barrier)
+      for (int idx = gt; idx < hc * m; idx += kGroupThreads) {
+        const int jh = idx / m, j = idx - jh * m, i = n + j;
+        const size_t o = (bh0 + jh) * cap + (slot_n + j) % cap;
+        const float g = logf(sg[jh * WMAX + i]);
+        sg[jh * WMAX + i] = g;
+        gring[o] = g;
+        bring[o] = sbeta[jh * WMAX + i];
+      }
       // ---- raw dots k_i.q_j and k_i.k_ej of every head and window entry i in
       //      [w0, n + j], in tasks (head, batch of CE entries) over the warps
       if (m > 0) {
@@ -743,65 +769,66 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         //      a pre-fold whose result the outputs read) and/or to the checkpoint.
         auto fold_tc = [&](int i0, int nf, int which, bool to_stage, bool to_global) {
           const float *fwv = fw + which * (kMaxW + 1);
-          const int KG = Y.umma_kg, KE = KG * 8;
+          constexpr int KG = 2, KE = 16;
           uint8_t *uA = reinterpret_cast<uint8_t *>(G + Y.umma);
           uint8_t *uB = uA + (DK / 8) * KG * 128;
-          const int partB = (HALF / 8) * KG * 128;
-          for (int idx = gt; idx < KE * (DK / 8); idx += kGroupThreads) {
-            const int i = idx / (DK / 8), cc = idx - i * (DK / 8);
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (i < nf) {
-              const int e = i0 + i;
-              if (e < n) {
-                val = *reinterpret_cast<const uint4 *>(kb + (size_t)e * DK + 8 * cc);
-              } else {   // a new token's k (bf16 values widened exactly): back to bf16
-                const float4 lo4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc);
-                const float4 hi4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc + 4);
-                const __nv_bfloat162 p0 = __floats2bfloat162_rn(lo4.x, lo4.y), p1 = __floats2bfloat162_rn(lo4.z, lo4.w);
-                const __nv_bfloat162 p2 = __floats2bfloat162_rn(hi4.x, hi4.y), p3 = __floats2bfloat162_rn(hi4.z, hi4.w);
-                val = make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
-                                 *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
-              }
-            }
-            *reinterpret_cast<uint4 *>(uA + umma::mn_offset(8 * cc, i, KG)) = val;
-          }
-          for (int p = lane; p < KE * RPW; p += 32) {
-            const int i = p >> 3, r8 = p & 7;
-            float x = 0.0f;
-            if (i < nf) {
-              const int e = i0 + i;
-              x = fwv[i] * (e < n ? wst[e * HALF + urow0 + r8] : wnew[(e - n) * RPW + r8]);
-            }
-            uint16_t xh, xm, xl;
-            umma::split3_bf16(x, xh, xm, xl);
-            const uint32_t off = umma::mn_offset(urow0 + r8, i, KG);
-            *reinterpret_cast<uint16_t *>(uB + off) = xh;
-            *reinterpret_cast<uint16_t *>(uB + partB + off) = xm;
-            *reinterpret_cast<uint16_t *>(uB + 2 * partB + off) = xl;
-          }
-          fence_proxy_async();   // operands written by this thread -> visible to the tensor core
-          umma::fence_before_sync();
-          named_sync(bar_id, kGroupThreads);
+          constexpr int partB = (HALF / 8) * KG * 128;
           const uint32_t tm = tmem_base + (uint32_t)(gi * HALF);
-          if (gt == 0) {
+          for (int blk = 0; blk < nf; blk += KE) {   // blocks of 16 entries, accumulated in TMEM
+            for (int idx = gt; idx < KE * (DK / 8); idx += kGroupThreads) {
+              const int i = idx / (DK / 8), cc = idx - i * (DK / 8);
+              uint4 val = make_uint4(0u, 0u, 0u, 0u);
+              if (blk + i < nf) {
+                const int e = i0 + blk + i;
+                if (e < n) {
+                  val = *reinterpret_cast<const uint4 *>(kb + (size_t)e * DK + 8 * cc);
+                } else {   // a new token's k (bf16 values widened exactly): back to bf16
+                  const float4 lo4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc);
+                  const float4 hi4 = *reinterpret_cast<const float4 *>(hk + (e - n) * DK + 8 * cc + 4);
+                  const __nv_bfloat162 p0 = __floats2bfloat162_rn(lo4.x, lo4.y), p1 = __floats2bfloat162_rn(lo4.z, lo4.w);
+                  const __nv_bfloat162 p2 = __floats2bfloat162_rn(hi4.x, hi4.y), p3 = __floats2bfloat162_rn(hi4.z, hi4.w);
+                  val = make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
+                                   *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
+                }
+              }
+              *reinterpret_cast<uint4 *>(uA + umma::mn_offset(8 * cc, i, KG)) = val;
+            }
+            for (int p = lane; p < KE * RPW; p += 32) {
+              const int i = p >> 3, r8 = p & 7;
+              float x = 0.0f;
+              if (blk + i < nf) {
+                const int e = i0 + blk + i;
+                x = fwv[blk + i] * (e < n ? wst[e * HALF + urow0 + r8] : wnew[(e - n) * RPW + r8]);
+              }
+              uint16_t xh, xm, xl;
+              umma::split3_bf16(x, xh, xm, xl);
+              const uint32_t off = umma::mn_offset(urow0 + r8, i, KG);
+              *reinterpret_cast<uint16_t *>(uB + off) = xh;
+              *reinterpret_cast<uint16_t *>(uB + partB + off) = xm;
+              *reinterpret_cast<uint16_t *>(uB + 2 * partB + off) = xl;
+            }
+            fence_proxy_async();   // operands written by this thread -> visible to the tensor core
+            umma::fence_before_sync();
+            named_sync(bar_id, kGroupThreads);
+            if (gt == 0) {
+              umma::fence_after_sync();
+              constexpr uint32_t idesc = umma::idesc_bf16_f32_mn(DK, HALF);
+              const uint64_t ad = umma::smem_desc_mn(smem_u32(uA), 128, KG * 128);
+              for (int part = 0; part < 3; ++part)
+                umma::mma_bf16(tm, ad, umma::smem_desc_mn(smem_u32(uB + part * partB), 128, KG * 128), idesc,
+                               part > 0 || blk > 0);
+              umma::commit(&mma_bar[gi]);
+            }
+            // the MMAs always complete: wait without the abort flag (bounded), so
+            // that TMEM and the operands are never reused under a running MMA
+            const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
+            ++mma_uses;
             umma::fence_after_sync();
-            constexpr uint32_t idesc = umma::idesc_bf16_f32_mn(DK, HALF);
-            for (int part = 0; part < 3; ++part)
-              for (int ks = 0; ks < KG / 2; ++ks)
-                umma::mma_bf16(tm, umma::smem_desc_mn(smem_u32(uA) + 256 * ks, 128, KG * 128),
-                               umma::smem_desc_mn(smem_u32(uB + part * partB) + 256 * ks, 128, KG * 128), idesc,
-                               part > 0 || ks > 0);
-            umma::commit(&mma_bar[gi]);
-          }
-          // the MMAs always complete: wait without the abort flag (bounded), so
-          // that TMEM is never released under a running MMA
-          const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
-          ++mma_uses;
-          umma::fence_after_sync();
-          if (!ok) {
-            *abort = 1;
-            failed = true;
-            return;
+            if (!ok) {
+              *abort = 1;
+              failed = true;
+              return;
+            }
           }
           const int q = gw & 3, c = 32 * q + lane, rh = (gw >> 2) * 32;
           float d[32];

@@ -18,6 +18,7 @@
 #include <algorithm>
 
 #include "rssm_device.cuh"
+#include "umma.cuh"
 
 namespace rssm {
 namespace {
@@ -188,6 +189,27 @@ __device__ __forceinline__ uint32_t e4m3x2_h2(uint32_t bits) {
   return h2bits(__half2(r));
 }
 
+// Folds of layers that read the fp32 checkpoint with bf16 inputs (headdim 64,
+// dstate 128) run on the tensor cores (tcgen05): the rank-l update of a head,
+// D^T[n][p] = sum_i B_i[n] (fw_i x_i[p]), is an M = 128 (dstate) x N = 64
+// (headdim) x K = l bf16 MMA chain with an fp32 accumulator in TMEM, 16 window
+// entries per block.  B rows are bf16 already (exact); each weighted x value
+// is split into three bf16 parts (hi, mid, lo; their sum is the fp32 value to
+// 2^-24), so the products are exact and only the fp32 accumulation rounds, as
+// on the CUDA cores.  The epilogue adds e^{G} h from the stage and stores.
+template <int P, int N, typename Tin, int RF>
+constexpr bool umma_fold() { return RF == RSSM_READ_FP32 && sizeof(Tin) == 2 && P == 64 && N == 128; }
+template <int P, int N, typename Tin, int RF>
+constexpr int umma_floats() { return umma_fold<P, N, Tin, RF>() ? (N / 8 + 3 * P / 8) * 2 * 128 / 4 : 0; }
+
+// Floats of one consumer group's shared-memory region (host and device agree):
+// B window and C rows, dt windows, B.C, per-head scalars, the f16 C of the
+// read-copy tensor-core path, then the fold operands (128-byte aligned).
+template <int P, int N, typename Tin, int RF, int MAXM>
+__host__ __device__ constexpr int group_mma_off(int L, int hc) {
+  return ((L + MAXM) * N + MAXM * N + hc * (L + MAXM) + MAXM * (L + MAXM) + hc * (MAXM * 32 + MAXM + 64 + 2) + 3) & ~3;
+}
+
 constexpr int kGroupWarps = 8;                  // consumer warps sharing one head
 constexpr int kGroups = 2;                      // consumer groups, alternating items
 constexpr int kGroupThreads = kGroupWarps * 32;
@@ -222,14 +244,19 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   constexpr int SB = scale_bytes<RF, P, N>();
   constexpr int RB = rc_row_bytes<RF, N>();
   constexpr int HS = MAXM * 32 + MAXM + 64 + 2;   // per-head scalars
+  constexpr bool kUmma = umma_fold<P, N, Tin, RF>();
+  constexpr uint32_t kTmemCols = kGroups * P;     // one P-column fp32 accumulator per consumer group
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
+  __shared__ uint64_t mma_bar[kGroups];           // tensor-core fold completion, one per group
+  __shared__ uint32_t tmem_base;
   // stage_use[s] = the use index u the producer last requested on stage s.  A
   // parity wait is exact only when the waiter is at most one phase ahead of
   // the barrier; a consumer group that skips the other group's item could be
   // further ahead, so it first waits for stage_use[s] == u.
   __shared__ int stage_use[kMaxStages];
   __shared__ int abort_flag;
+  __shared__ int never_set;                       // the timeout self-test waits for it
   // pair_inter[p % kPairSlots]: the heads of the CTA's items 2p and 2p + 1
   // alternate in the issue order (both items fold).  The producer decides it
   // before issuing the pair's first head, when no item of the pair has been
@@ -250,8 +277,9 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   // each group's region starts on a 128-byte boundary (float4 reads of B and C rows)
   constexpr bool kMma = mma_read<P, N, Tin, RF, MAXM>();
   constexpr int kUnitWarps = kMma ? 4 : kGroupWarps;   // warps that work on (and release) one head
-  const int mma_off = (WMAX * N + MAXM * N + hc * WMAX + MAXM * WMAX + hc * HS + 3) & ~3;
-  const int group_floats = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~31;
+  const int mma_off = group_mma_off<P, N, Tin, RF, MAXM>(L, hc);
+  const int umma_off = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~31;
+  const int group_floats = (umma_off + umma_floats<P, N, Tin, RF>() + 31) & ~31;
 
   const Tin *xin = reinterpret_cast<const Tin *>(a.in[0]);
   const Tin *Bin = reinterpret_cast<const Tin *>(a.in[1]);
@@ -273,10 +301,20 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       mbar_init(&empty[s], kUnitWarps);
       stage_use[s] = -1;
     }
+    for (int g = 0; g < kGroups; ++g) mbar_init(&mma_bar[g], 1);
     abort_flag = 0;
+    never_set = 0;
     mbar_fence_init();
   }
+  if constexpr (kUmma) {
+    if (warp == 0) {   // TMEM for both groups' fold accumulators; freed by warp 0 at the end
+      umma::alloc(&tmem_base, kTmemCols);
+      umma::relinquish();
+    }
+    umma::fence_before_sync();
+  }
   __syncthreads();
+  if constexpr (kUmma) umma::fence_after_sync();
 
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------------ producer
@@ -367,6 +405,11 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
   float *sCinv = sB + mma_off + N / 2;                                 // 1 / its power-of-two scale
   const int sub = kMma ? (gw >> 2) : 0;   // tensor-core path: 4-warp half of the group, alternate heads
   const int c0 = (lane % T::LPR) * 4;
+  int mma_uses = 0;   // completed tensor-core folds of this group (parity of mma_bar[gi])
+  if (a.stall_test && blockIdx.x == 0) {   // the timeout self-test: this CTA's waits run out
+    stall_on_unset_flag(&never_set, abort, a.wait_limit);
+    if (gt == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
+  }
   for (int k = gi; k < my_items; k += kGroups) {
     int b, g, chunk;
     item_of(k, b, g, chunk);
@@ -529,9 +572,111 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         const float *hs = ssc + jh * HS;
         const float *hcoef = hs, *hdec = hs + MAXM * 32, *hfw = hs + MAXM * 32 + MAXM;
         const float *hdecf = hfw + 64;
-        if (!wait_stage()) break;
+        {
+          const bool got = wait_stage();
+          // a tensor-core fold has group barriers inside: every warp must agree on doing it
+          if (kUmma && (pre || post)) {
+            if (named_sync_or(bar_id, kGroupThreads, !got)) break;
+          } else if (!got) {
+            break;
+          }
+        }
         const Stage stg{smem + s * stage_bytes, XOFF, XROW, n, L};
         bool done = false;
+        if constexpr (kUmma) {
+          // ---- tensor-core fold of the head by the whole group: h <- dec h +
+          //      sum_i x_i (fw_i B_i)^T over the window [i0, i0 + nf), as D^T[n][p] =
+          //      sum_i B_i[n] (fw_i x_i[p]), 16 entries per MMA block.  Operands:
+          //      A = the B rows (bf16, exact), B = three bf16 parts of fw_i x_i[p],
+          //      each warp writing its own 8 rows p.  The epilogue thread of state
+          //      column n adds dec h[p][n] from the stage for 32 rows p and stores the
+          //      result to the stage (to_stage: a pre-fold the outputs read) and/or
+          //      to the checkpoint.  Returns false if the MMA never completed.
+          auto fold_tc = [&](int i0, int nf, const float *fwv, float dec, bool to_stage, bool to_global) -> bool {
+            constexpr int KG = 2, KE = 16;
+            uint8_t *uA = reinterpret_cast<uint8_t *>(sB + umma_off);
+            uint8_t *uB = uA + (N / 8) * KG * 128;
+            constexpr int partB = (P / 8) * KG * 128;
+            const uint32_t tm = tmem_base + (uint32_t)(gi * P);
+            for (int blk = 0; blk < nf; blk += KE) {
+              for (int idx = gt; idx < KE * (N / 8); idx += kGroupThreads) {
+                const int i = idx / (N / 8), cc = idx - i * (N / 8);
+                uint4 val = make_uint4(0u, 0u, 0u, 0u);
+                if (blk + i < nf) {   // B row (bf16 values widened exactly in sB): back to bf16
+                  const float *src = sB + (i0 + blk + i) * N + 8 * cc;
+                  const float4 lo4 = *reinterpret_cast<const float4 *>(src);
+                  const float4 hi4 = *reinterpret_cast<const float4 *>(src + 4);
+                  const __nv_bfloat162 p0 = __floats2bfloat162_rn(lo4.x, lo4.y), p1 = __floats2bfloat162_rn(lo4.z, lo4.w);
+                  const __nv_bfloat162 p2 = __floats2bfloat162_rn(hi4.x, hi4.y), p3 = __floats2bfloat162_rn(hi4.z, hi4.w);
+                  val = make_uint4(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1),
+                                   *reinterpret_cast<const uint32_t *>(&p2), *reinterpret_cast<const uint32_t *>(&p3));
+                }
+                *reinterpret_cast<uint4 *>(uA + umma::mn_offset(8 * cc, i, KG)) = val;
+              }
+              for (int q = lane; q < KE * T::RPW; q += 32) {
+                const int i = q >> 3, r8 = q & 7, p = gw * T::RPW + r8;
+                const float x = blk + i < nf ? fwv[blk + i] * stg.x<Tin>(i0 + blk + i, p) : 0.0f;
+                uint16_t xh, xm, xl;
+                umma::split3_bf16(x, xh, xm, xl);
+                const uint32_t off = umma::mn_offset(p, i, KG);
+                *reinterpret_cast<uint16_t *>(uB + off) = xh;
+                *reinterpret_cast<uint16_t *>(uB + partB + off) = xm;
+                *reinterpret_cast<uint16_t *>(uB + 2 * partB + off) = xl;
+              }
+              fence_proxy_async();   // operands written by this thread -> visible to the tensor core
+              umma::fence_before_sync();
+              named_sync(bar_id, kGroupThreads);
+              if (gt == 0) {
+                umma::fence_after_sync();
+                constexpr uint32_t idesc = umma::idesc_bf16_f32_mn(N, P);
+                const uint64_t ad = umma::smem_desc_mn(smem_u32(uA), 128, KG * 128);
+                for (int part = 0; part < 3; ++part)
+                  umma::mma_bf16(tm, ad, umma::smem_desc_mn(smem_u32(uB + part * partB), 128, KG * 128), idesc,
+                                 part > 0 || blk > 0);
+                umma::commit(&mma_bar[gi]);
+              }
+              // the MMAs always complete: wait without the abort flag (bounded), so
+              // that TMEM and the operands are never reused under a running MMA
+              const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
+              ++mma_uses;
+              umma::fence_after_sync();
+              if (!ok) {
+                *abort = 1;
+                return false;
+              }
+            }
+            const int q = gw & 3, c = 32 * q + lane, rh = (gw >> 2) * 32;
+            float d[32];
+            umma::ld_32x32b_x32(tm + ((uint32_t)(32 * q) << 16) + (uint32_t)rh, d);
+            umma::fence_before_sync();
+            float *tile = reinterpret_cast<float *>(stg.base);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int p = rh + j;
+              const float val = fmaf(dec, tile[p * N + c], d[j]);
+              if (to_stage) tile[p * N + c] = val;
+              if (to_global) __stcs(hc_dst + (size_t)p * N + c, val);
+            }
+            return true;
+          };
+          bool okf = true;
+          if (pre) {   // the new tokens do not fit: fold the committed window first, into the stage
+            okf = fold_tc(0, n, hfw, hdecf[0], true, !post);
+            if (named_sync_or(bar_id, kGroupThreads, !okf)) break;   // the folded tile is complete
+          }
+          const int row0 = gw * T::RPW + lane / T::LPR;
+          float4 v[T::NLD];
+#pragma unroll
+          for (int l = 0; l < T::NLD; ++l)
+            v[l] = *reinterpret_cast<const float4 *>(stg.base + ((size_t)(row0 + l * T::RPI) * N + c0) * 4);
+          if (m > 0)
+            outputs<P, N, kGroupWarps, Tin, MAXM>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
+          if (post) {  // the decode filled the window: fold all of it
+            const bool okp = fold_tc(w0, n - w0 + 1, hfw + 32, hdecf[1], false, true);
+            if (named_sync_or(bar_id, kGroupThreads, !okp)) break;
+          }
+          done = true;
+        }
         if constexpr (kMma) {
           if (!pre && !post) {   // ---- tensor-core read: this warp's 16-row tile
             const int mt = gw & 3, g8 = lane >> 2, t4 = lane & 3;
@@ -672,7 +817,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     const bool any_abort = named_sync_or(bar_id, kGroupThreads, *abort != 0);
     if (any_abort) {
       if (gt == 0) atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
-      return;
+      break;   // every consumer thread still meets the others at the TMEM release below
     }
     if (!rp.refuse && gt == 0) {
       __threadfence();
@@ -698,6 +843,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         a.len[b] = n2;
         a.flushes[b] = fl;
       }
+    }
+  }
+  if constexpr (kUmma) {   // both groups are done with their accumulators
+    umma::fence_before_sync();
+    named_sync(3, kConsumers);
+    if (warp == 0) {
+      umma::fence_after_sync();
+      umma::dealloc(tmem_base, kTmemCols);
     }
   }
 }
@@ -778,10 +931,9 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t s) {
   const int hc = heads_per_cta(a.hpg);
   const size_t xrow = (size_t)P * sizeof(Tin);
   const size_t stage = ((size_t)tile_bytes<RF, P, N>() + scale_bytes<RF, P, N>() + (a.L + MAXM) * xrow + 127) & ~(size_t)127;
-  const size_t wmax = a.L + MAXM;
-  const size_t mma_off = (wmax * N + MAXM * N + hc * wmax + MAXM * wmax +
-                          (size_t)hc * (MAXM * 32 + MAXM + 64 + 2) + 3) & ~(size_t)3;
-  const size_t group_floats = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~(size_t)31;
+  const size_t mma_off = (size_t)group_mma_off<P, N, Tin, RF, MAXM>(a.L, hc);
+  const size_t umma_off = (mma_off + mma_floats<P, N, Tin, RF, MAXM>() + 31) & ~(size_t)31;
+  const size_t group_floats = (umma_off + umma_floats<P, N, Tin, RF>() + 31) & ~(size_t)31;
   const size_t fixed = kGroups * sizeof(float) * group_floats;
   // One CTA per SM (its 544 threads use the register file); as many stages as
   // fit in its shared memory, at most 5 for fp32 tiles (32 KiB each) and

@@ -17,6 +17,7 @@ struct rssm_handle {
   uint8_t *buf, *rc, *meta;
   const float *A, *D;
   long long wait_limit;
+  int stall_next;   // rssm_arm_timeout_test: the next replay launch takes the timeout path
 };
 
 namespace {
@@ -219,6 +220,8 @@ int launch_step(rssm_handle *h, int mode, int m, const void *const *in, void *ou
   a.mask = mask;
   int rc = plan_slots_for(h, a, s);
   if (rc) return rc;
+  a.stall_test = h->stall_next;   // armed self-test: this launch takes the timeout path
+  h->stall_next = 0;
   cudaError_t e = replay_launch(h, a, s);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");
@@ -299,6 +302,13 @@ int rssm_set_wait_limit(rssm_handle *h, long long cycles) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (cycles < 0) return fail(RSSM_ERR_INVALID_ARG, "wait limit must be >= 0 (0 = default)");
   h->wait_limit = cycles == 0 ? rssm::kDefaultWaitLimit : cycles;
+  return ok();
+}
+
+int rssm_arm_timeout_test(rssm_handle *h) {
+  if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
+  if (h->d.kind == RSSM_KDA) return fail(RSSM_ERR_UNSUPPORTED, "KDA replay launches have no waits to run out");
+  h->stall_next = 1;
   return ok();
 }
 
@@ -643,6 +653,8 @@ extern "C" int rssm_decode_step_static_scratch(rssm_handle *h, const void *const
   a.arrivals = arrivals;
   rc = plan_slots_for(h, a, (cudaStream_t)stream);
   if (rc) return rc;
+  a.stall_test = h->stall_next;
+  h->stall_next = 0;
   e = replay_launch(h, a, (cudaStream_t)stream);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) return cuda_fail(e, "replay kernel launch");

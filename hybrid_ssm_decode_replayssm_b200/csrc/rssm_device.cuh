@@ -315,11 +315,20 @@ __device__ __forceinline__ bool wait_flag_at_least(const int *flag, int value, v
   return true;
 }
 
+// The timeout self-test: wait (bounded) for a shared flag that nothing sets.
+// Sets *abort and returns once the limit runs out, like any other wait.
+__device__ __forceinline__ void stall_on_unset_flag(const int *never_set, volatile int *abort, long long limit) {
+  wait_flag_at_least(never_set, 1, abort, limit);
+}
+
 // Asynchronous 16-byte global -> shared copies (cp.async, L1 bypassed): issued
 // without holding registers; a thread's copies are complete after
 // cp_async_wait_all(), and visible to the other threads after a barrier.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src_gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");

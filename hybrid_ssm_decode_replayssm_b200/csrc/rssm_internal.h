@@ -46,6 +46,9 @@ struct StepArgs {
   // give-up limit (SM clock cycles) of the bounded waits on copies and on the
   // other warps; waits for the tensor cores and the final drain keep their own
   long long wait_limit;
+  // nonzero: the consumer warps of CTA 0 first wait for a flag that nothing
+  // sets, so that the wait runs out (rssm_arm_timeout_test)
+  int stall_test;
 };
 
 constexpr long long kDefaultWaitLimit = 2000000000LL;   // about a second at B200 clocks

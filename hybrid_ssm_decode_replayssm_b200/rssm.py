@@ -35,7 +35,7 @@ EXPORTED = [
     "rssm_decode_step_static_scratch", "rssm_conventional_step_quantized",
     "rssm_branch", "rssm_restore", "rssm_get_slots",
     "rssm_state_bytes", "rssm_export_state", "rssm_import_state", "rssm_get_lengths",
-    "rssm_set_wait_limit",
+    "rssm_set_wait_limit", "rssm_arm_timeout_test",
 ]
 RSSM_STATIC_SCRATCH_MAX_BATCH = 65536
 
@@ -86,6 +86,7 @@ def lib():
         L.rssm_get_bookkeeping.argtypes = [vp, vp, vp]
         L.rssm_get_lengths.argtypes = [vp, vp, vp, vp]
         L.rssm_set_wait_limit.argtypes = [vp, C.c_longlong]
+        L.rssm_arm_timeout_test.argtypes = [vp]
         L.rssm_branch.argtypes = [vp, vp, vp]
         L.rssm_restore.argtypes = [vp, vp, vp]
         L.rssm_get_slots.argtypes = [vp, vp, vp]

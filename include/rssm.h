@@ -210,6 +210,15 @@ int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev);
  * RSSM_ERR_INVALID_ARG.  Applies to the calls enqueued after it. */
 int rssm_set_wait_limit(rssm_handle *h, long long cycles);
 
+/* (No passage: a self-test of the timeout path.)  The next replay launch of
+ * this Mamba-2 or GDN handle (decode, verify, flush) has the consumer warps of
+ * its first CTA wait for a shared flag that nothing sets; the wait gives up
+ * after the handle's wait limit, sets RSSM_STATUS_TIMEOUT and the CTA ends
+ * early, exactly as a copy that never lands would make it.  Nothing faults or
+ * hangs; the launch's results are unspecified (call rssm_reset afterwards).
+ * KDA: RSSM_ERR_UNSUPPORTED (its kernel has no waits). */
+int rssm_arm_timeout_test(rssm_handle *h);
+
 /*
  * Decode one token per sequence [summary ¶2-3]: append its inputs to the
  * window and write its output, reading the checkpoint (or its read copy)

@@ -3,11 +3,13 @@
 Every wait of the replay kernels (a stage's asynchronous copies landing, the
 consumer warps releasing a stage) gives up after a limit, sets
 RSSM_STATUS_TIMEOUT and lets the launch end early with the device context
-intact.  The limit is a launch parameter (rssm_set_wait_limit); here it is set
-to 100 SM cycles, far below the time a stage's copies take to arrive, so the
-waits run out on purpose -- no fault, trap or endless loop is involved.  After
-rssm_reset (which also clears the per-sequence arrival counters an aborted
-launch may leave behind) the same layer decodes correctly again.
+intact.  The test arms the kernels' self-test (rssm_arm_timeout_test: the
+consumer warps of the first CTA wait for a shared flag that nothing sets) with
+a short limit (rssm_set_wait_limit, 20000 SM cycles), so that wait runs out on
+purpose -- no fault, trap or endless loop is involved -- and the rest of the
+CTA takes the same abort path a copy that never lands would.  After rssm_reset
+(which also clears the per-sequence arrival counters an aborted launch may
+leave behind) the same layer decodes correctly again.
 """
 import pytest
 import torch
@@ -38,7 +40,8 @@ def test_short_wait_limit_times_out_then_layer_recovers(kind):
         step = lambda S, t: og.step(S, t["q"], t["k"], t["v"], t["alpha"], t["beta"])
     L = rssm.lib()
     out = torch.empty(out_shape, device=DEV)
-    assert L.rssm_set_wait_limit(layer.handle, 100) == rssm.RSSM_OK
+    assert L.rssm_set_wait_limit(layer.handle, 20000) == rssm.RSSM_OK
+    assert L.rssm_arm_timeout_test(layer.handle) == rssm.RSSM_OK
     layer.decode_step(dev_inputs(tokens(0), keys), out)
     torch.cuda.synchronize()                      # the launch ended: no error, no hang
     assert layer.get_status(clear=True) & rssm.RSSM_STATUS_TIMEOUT
