@@ -41,6 +41,7 @@ def _worker(conn, kind, state0, params, out_scale):
     state = np.asarray(state0, np.float64)
     worst = {}
     failures = []
+    series = []
 
     def note(what, err, tol, tag):
         worst[what] = max(worst.get(what, 0.0), err)
@@ -72,6 +73,22 @@ def _worker(conn, kind, state0, params, out_scale):
                     note("output", scaled_error(y_gpu, y), tol, tag)
                 if ck_gpu is not None:
                     note("checkpoint", scaled_error(ck_gpu, state), tol, tag)
+            elif op == "decode_bound":
+                # per element |g - o| <= bound + slack * (|o| + rms(o)); keeps per-call
+                # max and mean-square of |g - o| / rms(o) and the worst ratio to the bound
+                _, tag, tok, y_gpu, bound, slack, ck_gpu, tol = msg
+                state, y = step(state, tok)
+                y_gpu = np.asarray(y_gpu, np.float64)
+                rms = np.sqrt(np.mean(y ** 2)) + 1e-300
+                err = np.abs(y_gpu - y)
+                allowed = np.asarray(bound, np.float64) + slack * (np.abs(y) + rms)
+                ratio = float(np.max(err / allowed))
+                worst["bound ratio"] = max(worst.get("bound ratio", 0.0), ratio)
+                if ratio > 1.0 and len(failures) < 5:
+                    failures.append(f"error bound exceeded at {tag}: ratio {ratio:.3f}")
+                series.append((float(np.max(err) / rms), float(np.mean((err / rms) ** 2))))
+                if ck_gpu is not None:
+                    note("checkpoint", scaled_error(ck_gpu, state), tol, tag)
             elif op == "verify":
                 _, tag, drafts, accept, y_gpu, fold_local, ck_gpu, tol = msg
                 if len(fold_local):   # a row folded before its drafts: checkpoint = committed state
@@ -84,10 +101,10 @@ def _worker(conn, kind, state0, params, out_scale):
             elif op == "narrow":
                 state = state[msg[1]]
             elif op == "done":
-                conn.send({"worst": worst, "failures": failures, "error": None})
+                conn.send({"worst": worst, "failures": failures, "series": series, "error": None})
                 return
     except Exception:   # report, do not hang the parent
-        conn.send({"worst": worst, "failures": failures, "error": traceback.format_exc()})
+        conn.send({"worst": worst, "failures": failures, "series": series, "error": traceback.format_exc()})
 
 
 class OracleWorkers:
@@ -132,6 +149,13 @@ class OracleWorkers:
             if a:
                 c.send(("decode", tag, {k: v[a] for k, v in tok.items()}, y, ck, tol))
 
+    def decode_bound(self, tag, tok, y_rows, bound_rows, slack, ck_rows, tol):
+        """As decode, with a per-element error bound (arrays at self.rows())."""
+        ys, bs, cks = self._split(y_rows), self._split(bound_rows), self._split(ck_rows)
+        for c, a, y, bd, ck in zip(self.conns, self.active, ys, bs, cks):
+            if a:
+                c.send(("decode_bound", tag, {k: v[a] for k, v in tok.items()}, y, bd, slack, ck, tol))
+
     def verify(self, tag, drafts, accept, y_rows, folded, ck_folded, tol):
         """drafts: full-batch [B, k, ...]; accept [B]; y_rows: GPU outputs at self.rows();
         folded: global rows that folded before their drafts this round, ck_folded
@@ -161,8 +185,11 @@ class OracleWorkers:
             self.active[i] = [a[j] for j in loc]
 
     def finish(self, timeout=1800):
-        """Collect every worker's worst errors and failures; returns (worst, failures)."""
+        """Collect every worker's worst errors and failures; returns (worst, failures).
+        The per-call error series of decode_bound calls, one list per worker, is
+        left in self.series."""
         worst, failures = {}, []
+        self.series = []
         for c, p in zip(self.conns, self.procs):
             c.send(("done",))
             if not c.poll(timeout):
@@ -174,6 +201,7 @@ class OracleWorkers:
             if r["error"]:
                 failures.append(r["error"])
             failures += r["failures"]
+            self.series.append(r.get("series", []))
             for k, v in r["worst"].items():
                 worst[k] = max(worst.get(k, 0.0), v)
         return worst, failures

@@ -231,7 +231,10 @@ def test_quantized_reads_within_first_window(fmt):
 
 @pytest.mark.parametrize("fmt", FMTS)
 def test_read_copy_keeps_fp32_recurrence(fmt):
-    """The fp32 checkpoint trajectory is bit-identical with and without a read copy,
+    """The fp32 checkpoint trajectory with and without a read copy agrees to fp32
+    rounding (both fold the same fp32 checkpoint and inputs; the fp32-read layer
+    folds on the tensor cores with an exact three-part split, the read-copy
+    layer on the CUDA cores, so only the order of the fp32 additions differs),
     and the read-copy output error stays within the quantisation bound."""
     shape = si.Mamba2Layer(4, 16, 64, 128, 4, window=16, dtype="bf16", state_std=0.1)
     lq, A, D, h0 = m2_layer(shape, read_fmt=fmt)
@@ -247,7 +250,7 @@ def test_read_copy_keeps_fp32_recurrence(fmt):
         ins = dev_inputs(tok, M2_KEYS)
         lq.decode_step(ins, yq)
         lf.decode_step(ins, yf)
-        assert torch.equal(lq.ckpt, lf.ckpt), f"fp32 checkpoints diverged at step {t}"
+        assert rel_err(lq.ckpt.cpu(), lf.ckpt.cpu()) < 1e-6, f"fp32 checkpoints diverged at step {t}"
         h_exact, y = _oracle_step(h_exact, tok, A, D)
         window_toks.append(tok64(tok))
         # bound: e^{G_t} sum_n |dh[p,n]| |C_n| with the per-element code-grid bound on dh
