@@ -254,13 +254,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
         if (t >= (c ? T1 : T0)) continue;
         const int Rc = c ? R1 : R0;
         const int s_ = (c ? R0 : 0) + t % Rc, u_ = t / Rc;
-        if (u_ == 0 || mbar_try_wait(&empty[s_], (uint32_t)((u_ - 1) & 1))) g = c;
+        if (u_ == 0 || mbar_test_wait(&empty[s_], (uint32_t)((u_ - 1) & 1))) g = c;
       }
-      if (g < 0) {
+      if (g < 0) {   // neither group has released a stage yet
         if (*abort || clock64() - idle_since > a.wait_limit) {
           timed_out = true;
           break;
         }
+        __nanosleep(20);
         continue;
       }
       idle_since = clock64();
