@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
       s = base + t % Rg;
       use = t / Rg;
     };
-    auto wait_stage = [&]() -> bool { return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit); };
+    auto wait_stage = [&]() -> bool { return warp_all(mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit)); };
     auto release_stage = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -822,7 +822,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
             }
             // the MMAs always complete: wait without the abort flag (bounded), so
             // that TMEM and the operands are never reused under a running MMA
-            const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
+            const bool ok = warp_all(mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit));
             ++mma_uses;
             umma::fence_after_sync();
             if (!ok) {
@@ -1190,6 +1190,7 @@ cudaError_t launch_conv(const ConvArgs &a, int in_dtype, cudaStream_t s) {
 bool gdn_supported(int R, int C) { return R == DV && C == DK; }
 
 cudaError_t gdn_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s) {
+  if (gdn_decode_fast_path(a, in_dtype, read_fmt)) return gdn_decode_step(a, s);
   if (in_dtype == RSSM_BF16) return dispatch_rf<__nv_bfloat16>(a, read_fmt, s);
   return dispatch_rf<float>(a, read_fmt, s);
 }

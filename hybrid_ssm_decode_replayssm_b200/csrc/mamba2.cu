@@ -524,14 +524,14 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
     const int seq_base = (k >> 1) * 2 * hc;
     int s = seq_base % stages, use = seq_base / stages;
     bool inter = false;
-    if (wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit)) {   // the pair's first head is issued
+    if (warp_all(wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit))) {   // the pair's first head is issued
       __threadfence_block();
       inter = *reinterpret_cast<volatile int *>(&pair_inter[(k >> 1) % kPairSlots]) != 0;
     }
     // wait until the producer has requested use `use` of stage s, then for the data
     auto wait_stage = [&]() -> bool {
-      if (!wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit)) return false;
-      return mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit);
+      if (!warp_all(wait_flag_at_least(&stage_use[s], use, abort, a.wait_limit))) return false;
+      return warp_all(mbar_wait_bounded(&full[s], (uint32_t)(use & 1), abort, a.wait_limit));
     };
     constexpr int hstep = kMma ? 2 : 1;   // heads taken by this warp: sub, sub + hstep, ...
     {
@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(kReplayThreads, 1)
               }
               // the MMAs always complete: wait without the abort flag (bounded), so
               // that TMEM and the operands are never reused under a running MMA
-              const bool ok = mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit);
+              const bool ok = warp_all(mbar_wait_bounded(&mma_bar[gi], (uint32_t)(mma_uses & 1), nullptr, kDefaultWaitLimit));
               ++mma_uses;
               umma::fence_after_sync();
               if (!ok) {

@@ -24,17 +24,33 @@ struct RowPlan {
   bool refuse, pre, post;
   unsigned bit;
 };
-__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
+// The pointers a plan is made from, loaded apart from their use so that a
+// warp can request the next item's while it works on the current one (they
+// cannot move before this CTA's own part of that sequence is done).
+struct RowRaw {
+  int st, n, src, dst, pend, mask;
+};
+__device__ __forceinline__ RowRaw load_row(const StepArgs &a, int b) {
+  RowRaw w;
+  w.st = a.start[b];
+  w.n = a.len[b];
+  w.src = a.slot ? a.slot[b] : b;
+  w.dst = a.dst ? a.dst[b] : b;
+  w.pend = a.pending[b];
+  w.mask = a.mask ? a.mask[b] : 1;
+  return w;
+}
+__device__ __forceinline__ RowPlan plan_from(const StepArgs &a, const RowRaw &w) {
   RowPlan r;
-  r.st = a.start[b];
-  r.n = a.len[b];
-  r.src = a.slot ? a.slot[b] : b;
-  r.dst = a.dst ? a.dst[b] : b;
-  const int pend = a.pending[b];
+  r.st = w.st;
+  r.n = w.n;
+  r.src = w.src;
+  r.dst = w.dst;
+  const int pend = w.pend;
   r.refuse = r.pre = r.post = false;
   r.bit = 0;
   if (a.mode == kFlush) {
-    if (a.mask != nullptr && a.mask[b] == 0) r.refuse = true;
+    if (w.mask == 0) r.refuse = true;
     else if (pend != 0) { r.refuse = true; r.bit = RSSM_STATUS_STATE; }
     else if (r.n == 0) r.refuse = true;
     else r.pre = true;
@@ -51,6 +67,7 @@ __device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) {
   }
   return r;
 }
+__device__ __forceinline__ RowPlan plan_row(const StepArgs &a, int b) { return plan_from(a, load_row(a, b)); }
 
 // ---------------------------------------------------------------- loads
 // The checkpoint is streamed once per call: keep it out of L1 and mark it
@@ -311,6 +328,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
   return true;
 }
+// Combine a per-lane wait result across the warp: every lane of the warp waits
+// on its own, and the warp goes on only if all of them succeeded, so a wait
+// that gives up in some lanes (an abort seen at slightly different times)
+// cannot split the warp before its collective operations (shuffles, named
+// barriers, tcgen05 loads).  Call with all 32 lanes.
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
 // Spin (bounded, abort-aware) until the shared int *flag reaches `value`.
 __device__ __forceinline__ bool wait_flag_at_least(const int *flag, int value, volatile int *abort,
                                                    long long limit = 2000000000LL) {
@@ -369,6 +393,21 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// The same copy with an L2 eviction-priority hint (a createpolicy value): the
+// checkpoint is streamed once per call, so its lines are marked evict-first and
+// the small window rows re-read every step stay in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_g2s_hint(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {

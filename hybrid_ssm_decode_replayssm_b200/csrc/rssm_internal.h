@@ -81,6 +81,10 @@ cudaError_t mamba2_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStrea
 // state stored in low precision and rounded again after every token
 cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s);
 cudaError_t gdn_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
+// The GDN decode serving path (one token, bf16 inputs, fp32 reads): its own
+// kernel with prologue warps and tensor-core folds (dr_decode.cu).
+bool gdn_decode_fast_path(const StepArgs &a, int in_dtype, int read_fmt);
+cudaError_t gdn_decode_step(const StepArgs &a, cudaStream_t s);
 cudaError_t gdn_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s);
 cudaError_t quantize_read_copy(const QuantArgs &a, int read_fmt, cudaStream_t s);
 cudaError_t rollback(int B, const int32_t *n_reject, int32_t *len, int32_t *pending,
