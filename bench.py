@@ -182,6 +182,7 @@ class Mamba2Work:
     name = "mamba2"
     keys = ("x", "B", "C", "dt")
     kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/mamba2.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/umma.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
 
@@ -232,7 +233,8 @@ class Mamba2Work:
 class GDNWork:
     name = "gdn"
     keys = ("q", "k", "v", "alpha", "beta")
-    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/gdn.cu",
+    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/dr_decode.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/umma.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
 
