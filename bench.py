@@ -283,7 +283,9 @@ class GDNWork:
 class KDAWork(GDNWork):
     """Kimi Delta Attention layer (per-channel gates) of the GDN serving shape."""
     name = "kda"
-    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/kda.cu",
+    kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/kda_decode.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/kda.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/umma.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
 

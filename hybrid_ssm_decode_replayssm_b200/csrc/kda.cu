@@ -6,8 +6,10 @@
 //   S_t = S_{t-1} Diag(alpha_t) + beta_t (v_t - S_{t-1} Diag(alpha_t) k_t) k_t^T,
 //   o_t = out_scale S_t q_t,  S in R^{dv x dk}.
 // Replay form over a window of entries 0..t on top of the checkpoint S_c, with
-// g = ln alpha per channel, seg(s,t) = sum_{s<r<=t} g_r (a direct suffix sum per
-// channel) and G_t = sum_{r<=t} g_r:
+// g = ln alpha per channel, seg(s,t) = sum_{s<r<=t} g_r and G_t = sum_{r<=t} g_r.
+// The ring keeps alpha itself, and e^{seg(s,t)} = prod_{s<r<=t} alpha_r is
+// formed as a running product per channel (the same value as the exponential
+// of the suffix sum, with no transcendental per entry):
 //   w_t = beta_t (v_t - S_c (e^{G_t} . k_t) - sum_{s<t} ((k_s . e^{seg(s,t)}) . k_t) w_s)
 //   o_t = out_scale (S_c (e^{G_t} . q_t) + sum_{s<=t} ((k_s . e^{seg(s,t)}) . q_t) w_s)
 //   fold: S_c <- S_c Diag(e^{G_t}) + sum_{s<=t} w_s (k_s . e^{seg(s,t)})^T
@@ -59,16 +61,16 @@ __device__ __forceinline__ void kda_fold(float4 (&S)[kRowsPerWarp], const float 
   }
 }
 
-// dec[s][c] = e^{seg(s,t)}, eG[c] = e^{G_t} from the log gates gw[0..t] (threads < KD, one channel each).
-__device__ __forceinline__ void kda_decays(const float *gw, float *dec, float *eG, int t) {
+// dec[s][c] = e^{seg(s,t)}, eG[c] = e^{G_t} from the gates aw[0..t] (threads < KD, one channel each).
+__device__ __forceinline__ void kda_decays(const float *aw, float *dec, float *eG, int t) {
   const int c = threadIdx.x;
   if (c < KD) {
-    float acc = 0.0f;
+    float acc = 1.0f;
     for (int s = t; s >= 0; --s) {
-      dec[s * KD + c] = expf(acc);
-      acc += gw[s * KD + c];
+      dec[s * KD + c] = acc;
+      acc *= aw[s * KD + c];
     }
-    eG[c] = expf(acc);
+    eG[c] = acc;
   }
 }
 
@@ -79,7 +81,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = a.L, cap = a.cap, wmax = L + 1;
   float *kw = sm;                   // [wmax][KD]  window k rows (fp32)
-  float *gw = kw + wmax * KD;       // [wmax][KD]  log gates
+  float *gw = kw + wmax * KD;       // [wmax][KD]  gates alpha
   float *ww = gw + wmax * KD;       // [wmax][KD]  w rows
   float *dec = ww + wmax * KD;      // [wmax][KD]  e^{seg(s, t)}
   float *qv = dec + wmax * KD, *vv = qv + KD, *eG = vv + KD, *uu = eG + KD, *yy = uu + KD;
@@ -138,9 +140,10 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   const Tin *kring = reinterpret_cast<const Tin *>(a.buf0) + (size_t)bh * cap * KD;
   Tin *kring_w = reinterpret_cast<Tin *>(a.buf0) + (size_t)bh * cap * KD;
   Tin *vring = reinterpret_cast<Tin *>(a.buf1) + (size_t)bh * cap * KD;
-  float *gring = a.buf2 + (size_t)bh * cap * KD;
+  float *gring = a.buf2 + (size_t)bh * cap * KD;   // alpha per channel
   float *bring = a.buf3 + (size_t)bh * cap;
-  float *wring = a.buf4 + (size_t)bh * cap * KD;
+  float *wring = a.buf4 + (size_t)bh * cap * KD;   // [2 halves][cap][KD / 2]
+  auto wslot = [&](size_t slot, int i) -> size_t { return ((size_t)(i / (KD / 2)) * cap + slot) * (KD / 2) + i % (KD / 2); };
 
   float *dst = a.hc + ((size_t)rp.dst * a.H + h) * KD * KD;   // where a fold writes
 
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
     const size_t slot = (size_t)((st + e) % cap);
     kw[idx] = to_f32<Tin>(kring[slot * KD + c]);
     gw[idx] = gring[slot * KD + c];
-    ww[idx] = wring[slot * KD + c];
+    ww[idx] = wring[wslot(slot, c)];
   }
   __syncthreads();
 
@@ -176,7 +179,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
     const size_t slot = (size_t)((st_new + t) % cap);
     const float beta = reinterpret_cast<const float *>(a.in[4])[bh];
     if (tid < KD) {
-      const float g = logf(ar);
+      const float g = ar;
       kw[t * KD + tid] = to_f32<Tin>(kr);
       gw[t * KD + tid] = g;
       qv[tid] = to_f32<Tin>(qr);
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
       for (int s = 0; s < t; ++s) r = fmaf(-Adot[s], ww[s * KD + i], r);
       const float w = beta * r;
       ww[t * KD + i] = w;
-      wring[slot * KD + i] = w;
+      wring[wslot(slot, i)] = w;
       float o = yy[i];
       for (int s = 0; s <= t; ++s) o = fmaf(Bdot[s], ww[s * KD + i], o);
       a.out[(size_t)bh * KD + i] = a.out_scale * o;
@@ -314,6 +317,7 @@ bool kda_supported(int R, int C) { return R == KD && C == KD; }
 
 cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s) {
   if (a.mode == kVerify) return cudaErrorNotSupported;
+  if (kda_decode_fast_path(a, in_dtype)) return kda_decode_step(a, s);
   return in_dtype == RSSM_BF16 ? launch_kda_step<__nv_bfloat16>(a, s) : launch_kda_step<float>(a, s);
 }
 

@@ -99,7 +99,7 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
     L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf [B,H,cap,dv]
     L->buf_off[2] = off; off = align256(off + B * H * cap * C * sizeof(float)); // g_buf [B,H,cap,dk]
     L->buf_off[3] = off; off = align256(off + B * H * cap * sizeof(float)); // beta_buf [B,H,cap]
-    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf [B,H,cap,dv]
+    L->buf_off[4] = off; off = align256(off + B * H * cap * R * sizeof(float)); // w_buf [B,H,2,cap,dv/2]
   } else {
     L->buf_off[0] = off; off = align256(off + B * H * cap * C * esz);      // k_buf [B,H,cap,dk]
     L->buf_off[1] = off; off = align256(off + B * H * cap * R * esz);      // v_buf [B,H,2,cap,dv/2]
@@ -110,6 +110,13 @@ void compute_layout(const rssm_layer_desc *d, rssm_layout *L, size_t *ckpt, size
   if (d->branching) {   // a copy of the ring regions for rssm_branch
     L->branch_scratch_off = off;
     off = align256(off + off);
+  }
+  if (d->kind == RSSM_KDA) {   // operands of the decode kernel's folds, per CTA
+    const size_t fs = rssm::kda_fold_scratch_bytes(*d);
+    if (fs) {
+      L->fold_scratch_off = off;
+      off = align256(off + fs);
+    }
   }
   *buf = off;
   if (d->read_fmt == RSSM_READ_FP32) {
@@ -166,6 +173,7 @@ rssm::StepArgs step_args(const rssm_handle *h, int mode, int m) {
     a.buf3 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[3]);
     a.buf4 = reinterpret_cast<float *>(h->buf + h->lay.buf_off[4]);
   }
+  if (h->lay.fold_scratch_off) a.fold_scratch = h->buf + h->lay.fold_scratch_off;
   a.start = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_start_off);
   a.len = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_len_off);
   a.pending = reinterpret_cast<int32_t *>(h->meta + h->lay.meta_pending_off);
@@ -453,9 +461,9 @@ int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream)
     const int outer[3] = {H, d.ngroups, H}, entry[3] = {d.headdim * esz, d.dstate * esz, 4};
     b.nreg = 3;
     for (int r = 0; r < 3; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
-  } else if (d.kind == RSSM_KDA) {   // k [H][cap][dk] | v [H][cap][dv] | g [H][cap][dk] fp32 | beta | w
-    const int outer[5] = {H, H, H, H, H};
-    const int entry[5] = {d.dstate * esz, d.headdim * esz, d.dstate * 4, 4, d.headdim * 4};
+  } else if (d.kind == RSSM_KDA) {   // k [H][cap][dk] | v [H][cap][dv] | g [H][cap][dk] fp32 | beta | w [2H][cap][dv/2]
+    const int outer[5] = {H, H, H, H, 2 * H};
+    const int entry[5] = {d.dstate * esz, d.headdim * esz, d.dstate * 4, 4, d.headdim / 2 * 4};
     b.nreg = 5;
     for (int r = 0; r < 5; ++r) b.outer[r] = outer[r], b.entry_bytes[r] = entry[r];
   } else {   // k [H][cap][dk] | v [2H][cap][dv/2] | g, beta [H][cap] | w [2H][cap][dv/2] fp32
@@ -507,7 +515,8 @@ struct Piece {
 int state_pieces(const rssm_handle *h, Piece (&p)[4]) {
   p[0] = {reinterpret_cast<uint8_t *>(h->ckpt), h->ckpt_bytes};
   p[1] = {h->rc, h->rc ? h->rc_bytes : 0};
-  p[2] = {h->buf, h->d.branching ? h->lay.branch_scratch_off : h->buf_bytes};
+  p[2] = {h->buf, h->d.branching ? h->lay.branch_scratch_off
+                  : h->lay.fold_scratch_off ? h->lay.fold_scratch_off : h->buf_bytes};
   p[3] = {h->meta, h->meta_bytes};
   return 4;
 }

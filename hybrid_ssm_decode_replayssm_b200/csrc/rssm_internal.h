@@ -36,6 +36,7 @@ struct StepArgs {
   // ring buffers (layer specific, see rssm.h)
   void *buf0, *buf1;     // Mamba-2: x_buf, B_buf     GDN: k_buf, v_buf
   float *buf2, *buf3, *buf4;  // Mamba-2: dt_buf     GDN: g_buf, beta_buf, w_buf
+  uint8_t *fold_scratch;      // KDA decode serving path: per-CTA fold operands (nullable)
   // per-call inputs / outputs
   const void *in[5];
   float *out;

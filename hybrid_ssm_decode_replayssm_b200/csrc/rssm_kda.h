@@ -1,4 +1,4 @@
-// Launchers of the KDA kernels (kda.cu) for the C-ABI host code.
+// Launchers of the KDA kernels (kda.cu, kda_decode.cu) for the C-ABI host code.
 #pragma once
 
 #include "rssm_internal.h"
@@ -8,6 +8,13 @@ namespace rssm {
 bool kda_supported(int R, int C);
 // decode (m = 1) and flush (m = 0); verify is not built for KDA
 cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s);
+// The decode serving path (one token, bf16 inputs): its own persistent kernel
+// with prologue warps and tensor-core folds (kda_decode.cu).
+bool kda_decode_fast_path(const StepArgs &a, int in_dtype);
+// Bytes of that kernel's per-CTA fold-operand scratch in the ring buffer (0 if
+// the kernel does not serve the descriptor).
+size_t kda_fold_scratch_bytes(const rssm_layer_desc &d);
+cudaError_t kda_decode_step(const StepArgs &a, cudaStream_t s);
 // fp32 state only
 cudaError_t kda_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s);
 

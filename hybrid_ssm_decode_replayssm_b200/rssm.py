@@ -54,7 +54,8 @@ class Layout(C.Structure):
                 ("meta_flushes_off", C.c_size_t), ("meta_arrivals_off", C.c_size_t),
                 ("meta_status_off", C.c_size_t), ("meta_slot_off", C.c_size_t),
                 ("meta_dst_off", C.c_size_t), ("meta_seen_off", C.c_size_t),
-                ("meta_work_off", C.c_size_t), ("branch_scratch_off", C.c_size_t)]
+                ("meta_work_off", C.c_size_t), ("branch_scratch_off", C.c_size_t),
+                ("fold_scratch_off", C.c_size_t)]
 
 
 _LIB = None

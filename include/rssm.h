@@ -133,8 +133,10 @@ typedef struct {
  *                 w_buf [B,H,2,cap,dv/2] fp32 (solved w_s, half-major; a cache
  *                 for reads, never used by a fold)
  *   buf, KDA:     k_buf [B,H,cap,dk] in_dtype | v_buf [B,H,cap,dv] in_dtype |
- *                 g_buf [B,H,cap,dk] fp32 (ln alpha per channel) |
- *                 beta_buf [B,H,cap] fp32 | w_buf [B,H,cap,dv] fp32 (solved w_s)
+ *                 a_buf [B,H,cap,dk] fp32 (alpha per channel; decays are
+ *                 running products of it) |
+ *                 beta_buf [B,H,cap] fp32 | w_buf [B,H,2,cap,dv/2] fp32 (solved
+ *                 w_s, half-major as for GDN)
  *   read copy, FP8 row: codes [B,H,R,C] uint8 | scales [B,H,R] fp32
  *   read copy, NVFP4:   codes [B,H,R,C/2] uint8 (element 2i in the low
  *                       nibble) | scales [B,H,R,C/16] uint8 (E4M3)
@@ -167,6 +169,8 @@ typedef struct {
   /* branching layers only (0 otherwise) */
   size_t meta_slot_off, meta_dst_off, meta_seen_off, meta_work_off;
   size_t branch_scratch_off;   /* in buf: a copy of the ring regions above */
+  size_t fold_scratch_off;     /* in buf, KDA with bf16 inputs: the decode
+                                  kernel's fold operands (0 if none) */
 } rssm_layout;
 
 typedef struct rssm_handle rssm_handle;

@@ -234,7 +234,7 @@ def test_state_io_checks_sizes():
         try:
             n = C.c_size_t()
             assert L.rssm_state_bytes(h, C.byref(n)) == rssm.RSSM_OK
-            ring = lay.branch_scratch_off if kw.get("branching") else buf
+            ring = lay.branch_scratch_off if kw.get("branching") else (lay.fold_scratch_off or buf)
             assert n.value == ck + rc + ring + meta
             assert L.rssm_export_state(h, fake, n.value + 1, None) == rssm.RSSM_ERR_INVALID_ARG
             assert L.rssm_import_state(h, None, n.value, None) == rssm.RSSM_ERR_INVALID_ARG
