@@ -14,15 +14,16 @@
 // The w_i of committed entries are kept in the ring (solved when their token
 // was decoded, against the same checkpoint).
 //
-// Roles of the 672 threads of a persistent CTA (one per SM):
+// Roles of the 768 threads of a persistent CTA (one per SM):
 //  * one producer warp: streams each unit -- half a head, 64 state rows (32 KiB
 //    fp32) and the committed w rows of those rows -- into a ring of
 //    shared-memory stages with 1-D TMA bulk copies, in the consumers' order;
-//  * four prologue warps: for each item (a sequence and a chunk of heads), one
-//    item ahead of the consumers, they append the new token to the rings and
-//    compute every head's window scalars (dots of the window k rows with q and
-//    k_e, segment decays as warp suffix sums, fold weights) into one of two
-//    item slots, so the consumers never wait on global memory for them;
+//  * seven prologue warps: for each item (a sequence and a chunk of heads), up
+//    to two items ahead of the consumers, they append the new token to the
+//    rings and compute every head's window scalars (dots of the window k rows
+//    with q and k_e, segment decays as warp suffix sums, fold weights) into one
+//    of three item slots, so the consumers never wait on global memory for
+//    them; a head is one task, and the tasks go to the warps in turn;
 //  * sixteen consumer warps: per unit, warp w owns rows 4w .. 4w+3, a row spread
 //    over 8 lanes (4 chunks of 4 columns); both matrix-vector products, the
 //    window sums, w_e and o_e; a fold runs on the tensor cores (tcgen05): the
@@ -37,7 +38,7 @@ namespace {
 
 constexpr int DK = 128, DV = 128, HALF = 64;
 constexpr int kCons = 16;                       // consumer warps
-constexpr int kPro = 4;                         // prologue warps
+constexpr int kPro = 7;                         // prologue warps (24 warps in all keep 80 registers)
 constexpr int kConsThreads = kCons * 32;
 constexpr int kThreads = (kCons + kPro + 1) * 32;
 constexpr int kProWarp0 = kCons, kProdWarp = kCons + kPro;
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
       mbar_init(&empty[s], kCons);
     }
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&slot_full[s], kPro);
+      mbar_init(&slot_full[s], hc);   // one arrival per head of the item
       mbar_init(&slot_empty[s], kCons);
     }
     mbar_init(&ops_bar, kCons);
@@ -143,8 +144,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
     if (lane != 0) return;
     int issued = 0;
     RowPlan rp{};
+    RowRaw nxt{};   // pointers of the next item, requested one item ahead
     int b = 0, chunk = 0;
     const uint64_t stream_once = l2_evict_first_policy();
+    if (my_items > 0) {
+      item_of(0, b, chunk);
+      nxt = load_row(a, b);
+    }
     for (int seq = 0; seq < my_items * units; ++seq) {
       const int k = seq / units, unit = seq - k * units, s = seq % stages, u = seq / stages;
       if (u > 0 && !mbar_wait_bounded(&empty[s], (uint32_t)((u - 1) & 1), abort, a.wait_limit)) {
@@ -153,7 +159,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
       }
       if (unit == 0) {
         item_of(k, b, chunk);
-        rp = plan_row(a, b);
+        rp = plan_from(a, nxt);
+        if (k + 1 < my_items) {
+          int bn, cn;
+          item_of(k + 1, bn, cn);
+          nxt = load_row(a, bn);
+        }
       }
       issued = seq + 1;
       if (rp.refuse) {
@@ -209,14 +220,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
         a.flushes[p.b] = fl;
       }
     };
+    // The item's heads are tasks t = k hc + jh, dealt to the prologue warps in
+    // turn (warp pw: tasks pw, pw + kPro, ...); a slot is full once every head
+    // of its item has arrived.  The task of head 0 also writes the item's plan
+    // and reports the slot's previous item done.
     bool pro_failed = false;
-    RowRaw nxt{};   // pointers of the next item, requested one item ahead
-    if (my_items > 0) {
+    const int ntasks = my_items * hc;
+    RowRaw nxt{};   // pointers of this warp's next task's sequence, requested one task ahead
+    if (pw < ntasks) {
       int b0, c0_;
-      item_of(0, b0, c0_);
+      item_of(pw / hc, b0, c0_);
       nxt = load_row(a, b0);
     }
-    for (int k = 0; k < my_items; ++k) {
+    for (int t = pw; t < ntasks; t += kPro) {
+      const int k = t / hc, jh = t - k * hc;
       const int sl = k % kSlots, use = k / kSlots;
       if (use > 0 && !warp_all(mbar_wait_bounded(&slot_empty[sl], (uint32_t)((use - 1) & 1), abort, a.wait_limit))) {
         atomicOr(a.status, (unsigned)RSSM_STATUS_TIMEOUT);
@@ -225,16 +242,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
       }
       float *slot = reinterpret_cast<float *>(smem + Y.slot_off + sl * Y.slot_bytes);
       SlotPlan *plan = reinterpret_cast<SlotPlan *>(slot);
-      if (use > 0 && pw == 0 && lane == 0) arrive_item(*plan);   // the slot's previous item is done
+      if (use > 0 && jh == 0 && lane == 0) arrive_item(*plan);   // the slot's previous item is done
       int b, chunk;
       item_of(k, b, chunk);
       const RowPlan rp = plan_from(a, nxt);
-      if (k + 1 < my_items) {
+      if (t + kPro < ntasks) {
         int bn, cn;
-        item_of(k + 1, bn, cn);
+        item_of((t + kPro) / hc, bn, cn);
         nxt = load_row(a, bn);
       }
-      if (pw == 0 && lane == 0) {
+      __syncwarp();
+      if (jh == 0 && lane == 0) {
         plan->b = b; plan->chunk = chunk; plan->st = rp.st; plan->n = rp.n; plan->src = rp.src;
         plan->dst = rp.dst; plan->refuse = rp.refuse; plan->pre = rp.pre; plan->post = rp.post;
         if (rp.refuse && rp.bit && chunk == 0) atomicOr(a.status, rp.bit);
@@ -242,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_decode_kernel(const StepArgs 
       if (!rp.refuse) {
         const int n = rp.n, st = rp.st, w0 = rp.pre ? n : 0;
         const int slot_n = (st + n) % cap;   // ring slot of the new entry
-        for (int jh = pw; jh < hc; jh += kPro) {
+        {
           const int h = chunk * hc + jh;
           const size_t bh = (size_t)b * a.H + h, tok = bh;   // one token per sequence
           float *hsl = slot + kPlanFloats + jh * HeadSlot::FLOATS;
