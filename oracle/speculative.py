@@ -15,7 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import gdn, mamba2
+from . import gdn, kda, mamba2
 
 
 def _draft(tokens, j):
@@ -43,6 +43,20 @@ def gdn_round(S, drafts, accept, out_scale=1.0):
     for j in range(k):
         tok = _draft(drafts, j)
         cur, o = gdn.step(cur, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"], out_scale)
+        states.append(cur)
+        outs.append(o)
+    new = np.stack([states[int(accept[b])][b] for b in range(S.shape[0])])
+    return np.stack(outs, axis=1), new
+
+
+def kda_round(S, drafts, accept, out_scale=1.0):
+    """S [B,H,dv,dk] committed; drafts {q,k,alpha[B,k,H,dk], v[B,k,H,dv], beta[B,k,H]}
+    (alpha one gate per key channel)."""
+    k = drafts["q"].shape[1]
+    states, outs, cur = [S], [], S
+    for j in range(k):
+        tok = _draft(drafts, j)
+        cur, o = kda.step(cur, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"], out_scale)
         states.append(cur)
         outs.append(o)
     new = np.stack([states[int(accept[b])][b] for b in range(S.shape[0])])

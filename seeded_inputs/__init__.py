@@ -33,7 +33,7 @@ __all__ = [
     "Mamba2Layer", "GDNLayer", "MAMBA2_TINY_F32", "MAMBA2_SERVING",
     "GDN_SERVING", "mamba2_params", "mamba2_checkpoint", "mamba2_tokens",
     "mamba2_drafts", "gdn_checkpoint", "gdn_tokens", "gdn_drafts",
-    "accept_counts", "torch_dtype",
+    "accept_counts", "torch_dtype", "kda_checkpoint", "kda_tokens", "kda_drafts",
 ]
 
 
@@ -208,21 +208,31 @@ def kda_checkpoint(layer: KDALayer, seed: int = 0) -> torch.Tensor:
     return torch.randn(shape, generator=_generator(seed, "kda.S0")) * layer.state_std
 
 
+def _kda_draw(layer: KDALayer, key, extra):
+    """q,k[B,*extra,H,dk], v[B,*extra,H,dv] (input dtype), alpha[B,*extra,H,dk] fp32
+    (one gate per key channel, the GDN recipe drawn per channel), beta[B,*extra,H] fp32."""
+    B, H, dk, dv = layer.batch, layer.nheads, layer.dk, layer.dv
+    dt_ = torch_dtype(layer.dtype)
+    q = torch.randn((B, *extra, H, dk), generator=_generator(*key, "q"))
+    k = torch.randn((B, *extra, H, dk), generator=_generator(*key, "k"))
+    q = q / torch.linalg.vector_norm(q, dim=-1, keepdim=True)
+    k = k / torch.linalg.vector_norm(k, dim=-1, keepdim=True)
+    v = torch.randn((B, *extra, H, dv), generator=_generator(*key, "v"))
+    za = torch.randn((B, *extra, H, dk), generator=_generator(*key, "alpha"))
+    zb = torch.randn((B, *extra, H), generator=_generator(*key, "beta"))
+    return {"q": q.to(dt_), "k": k.to(dt_), "v": v.to(dt_),
+            "alpha": torch.exp(-0.1 * F.softplus(za)).float(), "beta": torch.sigmoid(zb).float()}
+
+
 def kda_tokens(layer: KDALayer, step: int, seed: int = 0):
     """One decode token: q,k[B,H,dk], v[B,H,dv] (input dtype), alpha[B,H,dk] fp32 (one
     gate per key channel, the GDN recipe drawn per channel), beta[B,H] fp32."""
-    B, H, dk, dv = layer.batch, layer.nheads, layer.dk, layer.dv
-    key = (seed, "kda.tok", int(step))
-    dt_ = torch_dtype(layer.dtype)
-    q = torch.randn((B, H, dk), generator=_generator(*key, "q"))
-    k = torch.randn((B, H, dk), generator=_generator(*key, "k"))
-    q = q / torch.linalg.vector_norm(q, dim=-1, keepdim=True)
-    k = k / torch.linalg.vector_norm(k, dim=-1, keepdim=True)
-    v = torch.randn((B, H, dv), generator=_generator(*key, "v"))
-    za = torch.randn((B, H, dk), generator=_generator(*key, "alpha"))
-    zb = torch.randn((B, H), generator=_generator(*key, "beta"))
-    return {"q": q.to(dt_), "k": k.to(dt_), "v": v.to(dt_),
-            "alpha": torch.exp(-0.1 * F.softplus(za)).float(), "beta": torch.sigmoid(zb).float()}
+    return _kda_draw(layer, (seed, "kda.tok", int(step)), ())
+
+
+def kda_drafts(layer: KDALayer, rnd: int, k: int, seed: int = 0):
+    """k draft tokens: q,k[B,k,H,dk], v[B,k,H,dv], alpha[B,k,H,dk], beta[B,k,H]."""
+    return _kda_draw(layer, (seed, "kda.draft", int(rnd), int(k)), (k,))
 
 
 # ------------------------------------------------------------------ branching

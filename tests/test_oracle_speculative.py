@@ -4,7 +4,7 @@ import math
 
 import numpy as np
 
-from oracle import gdn, mamba2, speculative
+from oracle import gdn, kda, mamba2, speculative
 
 
 def test_mamba2_rollback_equals_accepted_prefix():
@@ -57,3 +57,45 @@ def test_gdn_rollback_equals_accepted_prefix():
     for b in range(B):
         Sb, _ = gdn.run(S0[b:b + 1], accepted[b])
         np.testing.assert_allclose(S[b], Sb[0], rtol=1e-12, atol=1e-12)
+
+
+def test_kda_rollback_equals_accepted_prefix():
+    rng = np.random.default_rng(13)
+    B, H, d, k, R = 2, 3, 4, 3, 6
+
+    def unit(v):
+        return v / np.linalg.norm(v, axis=-1, keepdims=True)
+    S0 = rng.standard_normal((B, H, d, d)) * 0.05
+    S = S0
+    accepted = [[] for _ in range(B)]
+    for r in range(R):
+        drafts = {"q": unit(rng.standard_normal((B, k, H, d))), "k": unit(rng.standard_normal((B, k, H, d))),
+                  "v": rng.standard_normal((B, k, H, d)),
+                  "alpha": np.exp(-0.1 * np.log1p(np.exp(rng.standard_normal((B, k, H, d))))),
+                  "beta": 1 / (1 + np.exp(-rng.standard_normal((B, k, H))))}
+        acc = rng.integers(0, k + 1, B)
+        outs, S = speculative.kda_round(S, drafts, acc)
+        for b in range(B):
+            seq = accepted[b] + [{n: drafts[n][b:b + 1, i] for n in drafts} for i in range(k)]
+            _, oo = kda.run(S0[b:b + 1], seq)
+            np.testing.assert_allclose(outs[b], oo[len(accepted[b]):, 0], rtol=1e-12, atol=1e-12)
+            accepted[b] += seq[len(accepted[b]): len(accepted[b]) + int(acc[b])]
+    for b in range(B):
+        Sb, _ = kda.run(S0[b:b + 1], accepted[b])
+        np.testing.assert_allclose(S[b], Sb[0], rtol=1e-12, atol=1e-12)
+
+
+def test_kda_round_with_equal_channel_gates_is_gdn_round():
+    """A per-channel gate that is the same on every channel is the gated delta rule's
+    scalar gate: the KDA round must give the GDN round's outputs and state."""
+    rng = np.random.default_rng(14)
+    B, H, d, k = 2, 2, 5, 4
+    S0 = rng.standard_normal((B, H, d, d)) * 0.05
+    a = np.exp(-0.1 * np.log1p(np.exp(rng.standard_normal((B, k, H)))))
+    drafts = {"q": rng.standard_normal((B, k, H, d)), "k": rng.standard_normal((B, k, H, d)) / d,
+              "v": rng.standard_normal((B, k, H, d)), "beta": 1 / (1 + np.exp(-rng.standard_normal((B, k, H))))}
+    acc = np.array([1, 3])
+    og, Sg = speculative.gdn_round(S0, dict(drafts, alpha=a), acc)
+    ok_, Sk = speculative.kda_round(S0, dict(drafts, alpha=np.repeat(a[..., None], d, axis=-1)), acc)
+    np.testing.assert_allclose(ok_, og, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(Sk, Sg, rtol=1e-12, atol=1e-12)
