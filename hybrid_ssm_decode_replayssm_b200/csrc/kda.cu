@@ -16,6 +16,12 @@
 // (. between vectors: elementwise).  The w_s of committed entries are kept in
 // the ring, so a decode reads S_c once and does two matrix-vector products.
 //
+// A verify call runs its k drafts through the same solve in order (draft j is
+// entry n + j, seeing S_c, the committed window and drafts 0 .. j-1) and leaves
+// them in the ring as pending entries with their w rows; a rollback keeps the
+// accepted prefix, whose w rows are then exactly those a decode of the same
+// tokens would have written.
+//
 // One CTA of 256 threads per (sequence, head).  The 128 x 128 fp32 tile sits in
 // registers: warp w holds rows 16w .. 16w+15, lane l columns 4l .. 4l+3.  The
 // window's k rows, log gates, cached w rows and decays sit in shared memory.
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   extern __shared__ __align__(16) float sm[];
   const int bh = blockIdx.x, b = bh / a.H, h = bh - b * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = a.L, cap = a.cap, wmax = L + 1;
+  const int L = a.L, cap = a.cap, wmax = L + (a.m > 1 ? a.m : 1);
   float *kw = sm;                   // [wmax][KD]  window k rows (fp32)
   float *gw = kw + wmax * KD;       // [wmax][KD]  gates alpha
   float *ww = gw + wmax * KD;       // [wmax][KD]  w rows
@@ -95,15 +101,19 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   float4 S[kRowsPerWarp];
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) S[i] = ld_stream(src + (size_t)(row0 + i) * KD + c0);
-  // and the new token's inputs (thread c < KD: channel / value row c)
+  // and the first new token's inputs (thread c < KD: channel / value row c)
   Tin kr{}, vr{}, qr{};
   float ar = 1.0f;
-  if (a.m == 1 && tid < KD) {
-    kr = reinterpret_cast<const Tin *>(a.in[1])[(size_t)bh * KD + tid];
-    vr = reinterpret_cast<const Tin *>(a.in[2])[(size_t)bh * KD + tid];
-    qr = reinterpret_cast<const Tin *>(a.in[0])[(size_t)bh * KD + tid];
-    ar = reinterpret_cast<const float *>(a.in[3])[(size_t)bh * KD + tid];
-  }
+  auto load_token = [&](int j) {   // token j of this call (decode: j = 0; verify: draft j)
+    if (tid < KD) {
+      const size_t tix = ((size_t)b * a.m + j) * a.H + h;
+      kr = reinterpret_cast<const Tin *>(a.in[1])[tix * KD + tid];
+      vr = reinterpret_cast<const Tin *>(a.in[2])[tix * KD + tid];
+      qr = reinterpret_cast<const Tin *>(a.in[0])[tix * KD + tid];
+      ar = reinterpret_cast<const float *>(a.in[3])[tix * KD + tid];
+    }
+  };
+  if (a.m >= 1) load_token(0);
 
   const RowPlan rp = plan_row(a, b);
   if (rp.refuse) {
@@ -129,6 +139,8 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
         n2 = 0;
         ++fl;
       }
+    } else if (a.mode == kVerify) {
+      a.pending[b] = a.m;   // the drafts are appended as pending entries
     }
     a.start[b] = st2;
     a.len[b] = n2;
@@ -173,11 +185,15 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
     n = 0;
   }
 
-  if (m == 1) {
-    // ---- the new token: entry t = n of the window, ring slot (st_new + n) % cap
-    const int t = n;
+  for (int j = 0; j < m; ++j) {
+    // ---- new token j (decode: the token; verify: draft j): entry t = n + j of the
+    //      window, ring slot (st_new + t) % cap; each solved against S_c and the
+    //      window entries before it
+    const int t = n + j;
     const size_t slot = (size_t)((st_new + t) % cap);
-    const float beta = reinterpret_cast<const float *>(a.in[4])[bh];
+    const size_t tix = ((size_t)b * m + j) * a.H + h;
+    const float beta = reinterpret_cast<const float *>(a.in[4])[tix];
+    if (j > 0) load_token(j);   // registers: the previous token ended on a barrier
     if (tid < KD) {
       const float g = ar;
       kw[t * KD + tid] = to_f32<Tin>(kr);
@@ -200,8 +216,8 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
       const float *other = isq ? qv : kw + t * KD;
       float acc = 0.0f;
 #pragma unroll
-      for (int j = 0; j < KD / 32; ++j) {
-        const int c = lane + 32 * j;
+      for (int jj = 0; jj < KD / 32; ++jj) {
+        const int c = lane + 32 * jj;
         acc = fmaf(kw[s * KD + c] * dec[s * KD + c], other[c], acc);
       }
       acc = warp_sum(acc);
@@ -235,11 +251,13 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
       wring[wslot(slot, i)] = w;
       float o = yy[i];
       for (int s = 0; s <= t; ++s) o = fmaf(Bdot[s], ww[s * KD + i], o);
-      a.out[(size_t)bh * KD + i] = a.out_scale * o;
+      a.out[tix * KD + i] = a.out_scale * o;
     }
     __syncthreads();
-    if (post) {   // the window is full: fold all of it
-      kda_fold(S, eG, kw, dec, ww, t, row0, c0);
+  }
+  if (m >= 1) {
+    if (post) {   // the decode filled the window: fold all of it
+      kda_fold(S, eG, kw, dec, ww, n, row0, c0);
 #pragma unroll
       for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
     } else if (pre) {
@@ -303,7 +321,7 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_conv_kernel(const ConvArgs
 template <typename Tin>
 cudaError_t launch_kda_step(const StepArgs &a, cudaStream_t s) {
   auto kern = kda_replay_kernel<Tin>;
-  const KdaSmem y{a.L + 1};
+  const KdaSmem y{a.L + (a.m > 1 ? a.m : 1)};   // the window and the new tokens
   const size_t smem = y.floats() * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -316,7 +334,6 @@ cudaError_t launch_kda_step(const StepArgs &a, cudaStream_t s) {
 bool kda_supported(int R, int C) { return R == KD && C == KD; }
 
 cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s) {
-  if (a.mode == kVerify) return cudaErrorNotSupported;
   if (kda_decode_fast_path(a, in_dtype)) return kda_decode_step(a, s);
   return in_dtype == RSSM_BF16 ? launch_kda_step<__nv_bfloat16>(a, s) : launch_kda_step<float>(a, s);
 }

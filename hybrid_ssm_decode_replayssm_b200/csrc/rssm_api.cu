@@ -315,7 +315,8 @@ int rssm_set_wait_limit(rssm_handle *h, long long cycles) {
 
 int rssm_arm_timeout_test(rssm_handle *h) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
-  if (h->d.kind == RSSM_KDA) return fail(RSSM_ERR_UNSUPPORTED, "KDA replay launches have no waits to run out");
+  if (h->d.kind == RSSM_KDA && rssm::kda_fold_scratch_bytes(h->d) == 0)
+    return fail(RSSM_ERR_UNSUPPORTED, "only the KDA decode serving kernel (bf16 inputs) has waits to run out");
   h->stall_next = 1;
   return ok();
 }
@@ -329,7 +330,6 @@ int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev, rssm_
 
 int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev, rssm_stream_t stream) {
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
-  if (h->d.kind == RSSM_KDA) return fail(RSSM_ERR_UNSUPPORTED, "verify is not built for KDA layers");
   if (h->d.max_draft < 1) return fail(RSSM_ERR_STATE, "handle was created with max_draft = 0");
   if (k < 1 || k > h->d.max_draft)
     return fail(RSSM_ERR_CAPACITY, "k = %d outside [1, max_draft = %d]", k, h->d.max_draft);

@@ -6,7 +6,7 @@
 namespace rssm {
 
 bool kda_supported(int R, int C);
-// decode (m = 1) and flush (m = 0); verify is not built for KDA
+// decode (m = 1), verify (m = k drafts) and flush (m = 0)
 cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s);
 // The decode serving path (one token, bf16 inputs): its own persistent kernel
 // with prologue warps and tensor-core folds (kda_decode.cu).

@@ -220,7 +220,9 @@ int rssm_set_wait_limit(rssm_handle *h, long long cycles);
  * after the handle's wait limit, sets RSSM_STATUS_TIMEOUT and the CTA ends
  * early, exactly as a copy that never lands would make it.  Nothing faults or
  * hangs; the launch's results are unspecified (call rssm_reset afterwards).
- * KDA: RSSM_ERR_UNSUPPORTED (its kernel has no waits). */
+ * KDA: only the decode serving kernel (bf16 inputs) waits, so only a decode of
+ * such a handle takes the path (a verify or flush launch just clears the armed
+ * test); a KDA handle with fp32 inputs gives RSSM_ERR_UNSUPPORTED. */
 int rssm_arm_timeout_test(rssm_handle *h);
 
 /*
@@ -249,7 +251,6 @@ int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev,
  * with a draft axis after the batch axis ([B,k,...]); out_dev is [B,k,H,P] /
  * [B,k,H,dv].  Output j is the output after drafts 0..j.  1 <= k <= max_draft.
  * A row with len + k > L is folded first (auto_flush; else CAPACITY, skipped).
- * KDA layers: RSSM_ERR_UNSUPPORTED.
  */
 int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev,
                 rssm_stream_t stream);

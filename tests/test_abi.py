@@ -216,7 +216,15 @@ def test_kda_descriptor_and_layout():
     assert L.rssm_create(C.byref(d_), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
     try:
         ins = (C.c_void_p * 5)(fake, fake, fake, fake, fake)
-        assert L.rssm_verify(h, 1, ins, fake, None) == rssm.RSSM_ERR_UNSUPPORTED
+        assert L.rssm_verify(h, 3, ins, fake, None) == rssm.RSSM_ERR_CAPACITY   # k > max_draft
+        assert L.rssm_verify(h, 0, ins, fake, None) == rssm.RSSM_ERR_CAPACITY
+        assert L.rssm_arm_timeout_test(h) == rssm.RSSM_OK   # bf16: the serving kernel has waits
+    finally:
+        L.rssm_destroy(h)
+    d_ = _desc(**dict(base, in_dtype=rssm.RSSM_F32))
+    assert L.rssm_create(C.byref(d_), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        assert L.rssm_arm_timeout_test(h) == rssm.RSSM_ERR_UNSUPPORTED
     finally:
         L.rssm_destroy(h)
 

@@ -11,7 +11,8 @@ window when it fills, and must give the recurrence's outputs and states:
 * the conventional per-token kernel (the in-run baseline) against the oracle;
 * explicit masked flush, restore to a position, and branching (rows sharing
   checkpoint slots) against the oracle's window rules;
-* verify is not built for KDA and says so.
+* speculative verify of k drafts with rollback to the accepted prefix against
+  the oracle's round (oracle.speculative.kda_round), and its refusals.
 """
 import numpy as np
 import pytest
@@ -20,8 +21,10 @@ import torch
 import seeded_inputs as si
 from gpu_common import DEV, KDA_KEYS, assert_close, dev_inputs, kda_layer, to64, tok64
 from hybrid_ssm_decode_replayssm_b200 import rssm
+from oracle import bookkeeping as obk
 from oracle import branch as ob
 from oracle import kda as ok
+from oracle import speculative as osp
 
 pytestmark = pytest.mark.gpu
 
@@ -100,10 +103,65 @@ def test_flush_restore_branch_against_oracle():
         assert_close(layer.checkpoint_rows().cpu(), rows.checkpoint(), TOL["bf16"], f"{op} {i}: checkpoints")
 
 
-def test_verify_is_not_built_for_kda():
-    shape = si.KDALayer(batch=2, nheads=4, dk=128, dv=128, window=8, dtype="bf16")
-    layer, _ = kda_layer(shape)
-    tok = si.kda_tokens(shape, 0)
-    with pytest.raises(rssm.RSSMError) as e:
-        layer.verify(1, dev_inputs(tok, KDA_KEYS), torch.empty((2, 1, 4, 128), device=DEV))
-    assert e.value.code == rssm.RSSM_ERR_UNSUPPORTED
+def _bk(layer):
+    return [list(map(int, r)) for r in layer.get_bookkeeping().cpu().numpy()]
+
+
+@pytest.mark.parametrize("k,L,dtype", [(1, 1, "f32"), (3, 4, "f32"), (4, 16, "bf16"), (8, 8, "bf16"),
+                                       (8, 32, "f32")])
+def test_verify_rollback(k, L, dtype):
+    """Verify rounds of k seeded drafts with seeded acceptance, decode steps in
+    between: every draft output is the recurrence's output after drafts 0..j,
+    the accepted prefix becomes committed window entries (their cached w rows
+    are what later decodes and folds read), and a round that does not fit is
+    folded first.  With bf16 inputs the decodes in between run on the serving
+    kernel, which reads the ring the verify kernel wrote."""
+    shape = si.KDALayer(batch=5, nheads=2, dk=128, dv=128, window=L, dtype=dtype, state_std=0.05)
+    layer, S0 = kda_layer(shape, seed=k, max_draft=k)
+    S = to64(S0)
+    book = obk.WindowBook(5, L, int(layer.layout.cap))
+    o = torch.empty(5, 2, 128, device=DEV)
+    outk = torch.empty(5, k, 2, 128, device=DEV)
+    for r in range(10):
+        drafts = si.kda_drafts(shape, r, k, seed=k)
+        acc = si.accept_counts(5, r, k, seed=k)
+        layer.verify(k, dev_inputs(drafts, KDA_KEYS), outk)
+        book.verify(k)
+        want, S_next = osp.kda_round(S, tok64(drafts), acc.numpy())
+        assert_close(outk.cpu(), want, TOL[dtype], f"verify round {r}")
+        n_reject = (k - acc).to(torch.int32)
+        layer.rollback(n_reject.to(DEV))
+        book.rollback(n_reject.tolist())
+        S = S_next
+        assert _bk(layer) == [list(x) for x in book.snapshot()], f"pointers after round {r}"
+        if r % 2 == 1:
+            tok = si.kda_tokens(shape, 500 + r, seed=k)
+            layer.decode_step(dev_inputs(tok, KDA_KEYS), o)
+            book.decode()
+            S, y = _step(S, tok64(tok))
+            assert_close(o.cpu(), y, TOL[dtype], f"decode after round {r}")
+    layer.flush()
+    book.flush()
+    assert_close(layer.ckpt.cpu(), S, TOL[dtype], "checkpoint after the rounds")
+    assert _bk(layer) == [list(x) for x in book.snapshot()]
+    assert layer.get_status() == 0
+
+
+def test_verify_refusals():
+    """A verify over a row whose drafts are still pending sets STATE; with
+    auto_flush off, drafts that do not fit in the window set CAPACITY.  Refused
+    rows keep their pointers and their checkpoint."""
+    shape = si.KDALayer(batch=2, nheads=4, dk=128, dv=128, window=4, dtype="bf16", state_std=0.05)
+    layer, S0 = kda_layer(shape, auto_flush=False, max_draft=3)
+    outk = torch.empty(2, 3, 4, 128, device=DEV)
+    layer.verify(3, dev_inputs(si.kda_drafts(shape, 0, 3), KDA_KEYS), outk)
+    before = _bk(layer)
+    layer.verify(3, dev_inputs(si.kda_drafts(shape, 1, 3), KDA_KEYS), outk)
+    assert layer.get_status(clear=True) == rssm.RSSM_STATUS_STATE
+    assert _bk(layer) == before
+    layer.rollback(torch.zeros(2, dtype=torch.int32, device=DEV))   # 3 committed of 4
+    before = _bk(layer)
+    layer.verify(2, dev_inputs(si.kda_drafts(shape, 2, 2), KDA_KEYS), outk[:, :2].contiguous())
+    assert layer.get_status(clear=True) == rssm.RSSM_STATUS_CAPACITY
+    assert _bk(layer) == before
+    assert_close(layer.ckpt.cpu(), to64(S0), 0.0, "checkpoint untouched")

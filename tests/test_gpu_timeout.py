@@ -15,15 +15,17 @@ import pytest
 import torch
 
 import seeded_inputs as si
-from gpu_common import DEV, GDN_KEYS, M2_KEYS, assert_close, dev_inputs, gdn_layer, m2_layer, tok64
+from gpu_common import (DEV, GDN_KEYS, KDA_KEYS, M2_KEYS, assert_close, dev_inputs, gdn_layer, kda_layer,
+                        m2_layer, tok64)
 from hybrid_ssm_decode_replayssm_b200 import rssm
 from oracle import gdn as og
+from oracle import kda as ok
 from oracle import mamba2 as om
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("kind", ["mamba2", "gdn"])
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
 def test_short_wait_limit_times_out_then_layer_recovers(kind):
     if kind == "mamba2":
         shape = si.Mamba2Layer(batch=64, nheads=16, headdim=64, dstate=128, ngroups=2, window=16,
@@ -32,12 +34,18 @@ def test_short_wait_limit_times_out_then_layer_recovers(kind):
         tokens = lambda t: si.mamba2_tokens(shape, t, seed=4)
         keys, out_shape = M2_KEYS, (64, 16, 64)
         step = lambda S, t: om.step(S, t["x"], t["B"], t["C"], t["dt"], A, D)
-    else:
+    elif kind == "gdn":
         shape = si.GDNLayer(batch=64, nheads=8, dk=128, dv=128, window=16, dtype="bf16", state_std=0.05)
         layer, h0 = gdn_layer(shape, seed=4)
         tokens = lambda t: si.gdn_tokens(shape, t, seed=4)
         keys, out_shape = GDN_KEYS, (64, 8, 128)
         step = lambda S, t: og.step(S, t["q"], t["k"], t["v"], t["alpha"], t["beta"])
+    else:   # the KDA decode serving kernel (bf16 inputs)
+        shape = si.KDALayer(batch=64, nheads=8, dk=128, dv=128, window=16, dtype="bf16", state_std=0.05)
+        layer, h0 = kda_layer(shape, seed=4)
+        tokens = lambda t: si.kda_tokens(shape, t, seed=4)
+        keys, out_shape = KDA_KEYS, (64, 8, 128)
+        step = lambda S, t: ok.step(S, t["q"], t["k"], t["v"], t["alpha"], t["beta"])
     L = rssm.lib()
     out = torch.empty(out_shape, device=DEV)
     assert L.rssm_set_wait_limit(layer.handle, 20000) == rssm.RSSM_OK
