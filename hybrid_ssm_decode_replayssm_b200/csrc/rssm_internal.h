@@ -78,6 +78,10 @@ struct QuantArgs {
 
 // Launchers return cudaGetLastError() of their launch.
 cudaError_t mamba2_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
+// Decode of read-copy layers (one token, bf16 inputs, headdim 64, dstate 128):
+// its own kernel without a stage pipeline (m2_rc_decode.cu).
+bool m2_rc_decode_path(const StepArgs &a, int in_dtype, int read_fmt);
+cudaError_t m2_rc_decode_step(const StepArgs &a, int read_fmt, cudaStream_t s);
 // state_fmt: RSSM_READ_FP32 (fp32 state), or the FP8 row / NVFP4 format of a
 // state stored in low precision and rounded again after every token
 cudaError_t mamba2_conventional(const ConvArgs &a, int in_dtype, int state_fmt, cudaStream_t s);
