@@ -21,7 +21,8 @@
 // m2_common.cuh).  The CTA's prologue stages the window: B rows (fp32), C,
 // the dt windows, B.C, the window scalars and every head's x rows, with the
 // ring appends.  Rows that fold this call (window full, or the token does not
-// fit) take the CUDA-core path of the general kernel, 8 rows at a time.
+// fit) take the CUDA-core path of the general kernel, 4 rows at a time.  At
+// 64 registers a thread, four CTAs (32 warps) share an SM.
 #include "m2_common.cuh"
 #include "rssm_device.cuh"
 
@@ -51,10 +52,11 @@ struct RcSmem {
 };
 
 // The codes and scales a lane needs for one batch of m-tiles (16 rows each) of
-// a head: NVFP4 four m-tiles (the whole head), FP8 two.
+// a head: NVFP4 two m-tiles, FP8 one (16 registers of codes either way, so that
+// four CTAs fit on an SM).
 template <int RF>
 struct RcCodes {
-  static constexpr int kTiles = RF == RSSM_READ_NVFP4 ? 4 : 2;
+  static constexpr int kTiles = RF == RSSM_READ_NVFP4 ? 2 : 1;
   static constexpr int kBatches = 4 / kTiles;
   uint4 q[8];
   uint32_t s[8];
@@ -93,9 +95,10 @@ __device__ __forceinline__ void load_batch(RcCodes<RF> &c, const uint8_t *codes,
 // (copy . C) of row 16 mt + (lane & 15) for m-tile k of the batch (the scale of
 // C not yet removed), from eight m16n8k16 steps; C sits in column 0 of B.
 template <int RF>
-__device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint32_t (&bfr)[16], int lane) {
+__device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint2 *cfrag, int lane) {
   float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   uint32_t af[4];
+  const bool holder = (lane >> 2) == 0;   // column 0 of B: lanes 0..3
   if constexpr (RF == RSSM_READ_NVFP4) {
     const uint32_t wa[4] = {c.q[2 * k].x, c.q[2 * k].y, c.q[2 * k].z, c.q[2 * k].w};
     const uint32_t wb[4] = {c.q[2 * k + 1].x, c.q[2 * k + 1].y, c.q[2 * k + 1].z, c.q[2 * k + 1].w};
@@ -110,7 +113,8 @@ __device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint
       af[1] = e2m1x2_scaled(wb[ks >> 1] >> sh, scb);
       af[2] = e2m1x2_scaled(wa[ks >> 1] >> (sh + 8), sca);
       af[3] = e2m1x2_scaled(wb[ks >> 1] >> (sh + 8), scb);
-      mma_16816(d, af, bfr[2 * ks], bfr[2 * ks + 1]);
+      const uint2 bv = holder ? cfrag[8 * (lane & 3) + ks] : make_uint2(0u, 0u);
+      mma_16816(d, af, bv.x, bv.y);
     }
   } else {
     const uint32_t wa[8] = {c.q[4 * k].x, c.q[4 * k].y, c.q[4 * k].z, c.q[4 * k].w,
@@ -123,7 +127,8 @@ __device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint
       af[1] = e4m3x2_h2(wb[ks]);
       af[2] = e4m3x2_h2(wa[ks] >> 16);
       af[3] = e4m3x2_h2(wb[ks] >> 16);
-      mma_16816(d, af, bfr[2 * ks], bfr[2 * ks + 1]);
+      const uint2 bv = holder ? cfrag[8 * (lane & 3) + ks] : make_uint2(0u, 0u);
+      mma_16816(d, af, bv.x, bv.y);
     }
     d[0] *= __uint_as_float(c.s[2 * k]);
     d[2] *= __uint_as_float(c.s[2 * k + 1]);
@@ -136,9 +141,9 @@ __device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint
 }
 
 template <int RF>
-__global__ void __launch_bounds__(kRcThreads, 2) m2_rc_decode_kernel(const StepArgs a, const int hc) {
+__global__ void __launch_bounds__(kRcThreads, 4) m2_rc_decode_kernel(const StepArgs a, const int hc) {
   using Tin = __nv_bfloat16;
-  using T = Tile<RP, RN, 8>;   // the fold path's 8-row groups: a lane holds 4 columns of 8 rows
+  using T = Tile<RP, RN, 16>;   // the fold path's 4-row groups: a lane holds 4 columns of 4 rows
   using Codes = RcCodes<RF>;
   constexpr int TB = tile_bytes<RF, RP, RN>();
   constexpr int RB = rc_row_bytes<RF, RN>();
@@ -306,14 +311,7 @@ __global__ void __launch_bounds__(kRcThreads, 2) m2_rc_decode_kernel(const StepA
   //      window scalars itself: output coefficients e^{A seg(i, n)} dt_i (B_i . C)
   //      over [w0, n] and e^{A G}; fold weights e^{A seg(i, last)} dt_i and the
   //      decay of each folded window.  Segment sums are warp suffix sums of dt.
-  uint32_t bfr[16];   // C (f16) in column 0 of the B fragments, permuted k order: C[32 t4 + 4 ks .. + 3]
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    uint2 v = make_uint2(0u, 0u);
-    if ((lane >> 2) == 0) v = *reinterpret_cast<const uint2 *>(sCh + 32 * (lane & 3) + 4 * ks);
-    bfr[2 * ks] = v.x;
-    bfr[2 * ks + 1] = v.y;
-  }
+  const uint2 *cfrag = reinterpret_cast<const uint2 *>(sCh);   // C (f16): the B fragments, C[32 t4 + 4 ks .. + 3]
   const float cinv = *sCinv;
   for (int jh = warp; jh < hc; jh += kRcWarps) {
     const int h = h0 + jh;
@@ -339,31 +337,33 @@ __global__ void __launch_bounds__(kRcThreads, 2) m2_rc_decode_kernel(const StepA
 #pragma unroll
         for (int q = 0; q < 2; ++q) ws[q] = fmaf(ci, stg.x<Tin>(w0 + i, lane + 32 * q), ws[q]);
       }
-      // tensor-core read of the copy, batch by batch (NVFP4: one batch of four
-      // 16-row m-tiles; FP8: two of two); the next batch, or the next head's
+      // tensor-core read of the copy, batch by batch (NVFP4: two batches of two
+      // 16-row m-tiles; FP8: four of one); the next batch, or the next head's
       // first, is requested as soon as this one's codes are used
 #pragma unroll
       for (int bi = 0; bi < Codes::kBatches; ++bi) {   // cq holds batch bi of this head
         float hcv[Codes::kTiles];
 #pragma unroll
-        for (int k = 0; k < Codes::kTiles; ++k) hcv[k] = tile_hc<RF>(cq, k, bfr, lane);
+        for (int k = 0; k < Codes::kTiles; ++k) hcv[k] = tile_hc<RF>(cq, k, cfrag, lane);
         if (bi + 1 < Codes::kBatches) {
           load_batch<RF>(cq, a.rc_codes + sbh * TB, a.rc_scales, sbh * RP, bi + 1, lane);
         } else if (jh + kRcWarps < hc) {
           const size_t nbh = sbh + kRcWarps;
           load_batch<RF>(cq, a.rc_codes + nbh * TB, a.rc_scales, nbh * RP, 0, lane);
         }
-        // lane l takes rows 32 q + l of the batch's m-tile pairs: m-tile 2 q + (l >= 16)
-#pragma unroll
-        for (int q = 0; q < Codes::kTiles / 2; ++q) {
-          const int rq = Codes::kTiles == 4 ? q : bi;   // which 32-row half of the head
-          const int row = 32 * rq + lane;
-          const float hcr = lane < 16 ? hcv[2 * q] : hcv[2 * q + 1];
-          a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcr * cinv, ws[rq]));
+        if constexpr (Codes::kTiles == 2) {   // rows 32 bi + lane: m-tile 2 bi + (lane >= 16)
+          const int row = 32 * bi + lane;
+          const float hcr = lane < 16 ? hcv[0] : hcv[1];
+          a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcr * cinv, ws[bi]));
+        } else {   // rows 16 bi + (lane & 15), written by lanes 0..15
+          const int row = 16 * bi + (lane & 15);
+          const float wsr = __shfl_sync(kFull, ws[bi >> 1], row & 31);
+          if (lane < 16)
+            a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcv[0] * cinv, wsr));
         }
       }
     } else {
-      // ---- a fold this call: the general kernel's CUDA-core path, 8 rows at a
+      // ---- a fold this call: the general kernel's CUDA-core path, 4 rows at a
       //      time, with this head's scalars in its slot of shared memory
       float *hs = ssc + jh * kHS;
       hs[lane] = coef;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kRcThreads, 2) m2_rc_decode_kernel(const StepA
           float4 f[T::NLD];
 #pragma unroll
           for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_src + (size_t)(row0 + l) * RN + c0);
-          fold_tile<RP, RN, 8, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
+          fold_tile<RP, RN, 16, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
 #pragma unroll
           for (int l = 0; l < T::NLD; ++l) {
             const int row = row0 + l;
@@ -404,13 +404,13 @@ __global__ void __launch_bounds__(kRcThreads, 2) m2_rc_decode_kernel(const StepA
           for (int l = 0; l < T::NLD; ++l)
             v[l] = load_read_copy4<RF>(rc_src + (size_t)(row0 + l) * RB, a.rc_scales, sbh * RP + row0 + l, RN, c0);
         }
-        outputs<RP, RN, 8, Tin, 1>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
+        outputs<RP, RN, 16, Tin, 1>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
         if (post) {   // the decode filled the window: fold it (after a pre-fold, from what that stored)
           const float *fsrc = pre ? hc_dst : hc_src;
           float4 f[T::NLD];
 #pragma unroll
           for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(fsrc + (size_t)(row0 + l) * RN + c0);
-          fold_tile<RP, RN, 8, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
+          fold_tile<RP, RN, 16, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
 #pragma unroll
           for (int l = 0; l < T::NLD; ++l) {
             const int row = row0 + l;
