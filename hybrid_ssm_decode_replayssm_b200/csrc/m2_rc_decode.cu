@@ -20,9 +20,11 @@
 // with C on the tensor cores (mma.sync m16n8k16, f16 in, fp32 out; exact, see
 // m2_common.cuh).  The CTA's prologue stages the window: B rows (fp32), C,
 // the dt windows, B.C, the window scalars and every head's x rows, with the
-// ring appends.  Rows that fold this call (window full, or the token does not
-// fit) take the CUDA-core path of the general kernel, 4 rows at a time.  At
-// 64 registers a thread, four CTAs (32 warps) share an SM.
+// ring appends.  A row that folds this call does so on the CUDA cores, 4 state
+// rows at a time (fp32 read, rank-l update, fp32 store, new copy); its outputs
+// come from the copy as well: the old one when the window fills with this
+// token, the new one when the token did not fit and the window was folded
+// first.  At 64 registers a thread, four CTAs (32 warps) share an SM.
 #include "m2_common.cuh"
 #include "rssm_device.cuh"
 
@@ -143,7 +145,7 @@ __device__ __forceinline__ float tile_hc(const RcCodes<RF> &c, int k, const uint
 template <int RF>
 __global__ void __launch_bounds__(kRcThreads, 4) m2_rc_decode_kernel(const StepArgs a, const int hc) {
   using Tin = __nv_bfloat16;
-  using T = Tile<RP, RN, 16>;   // the fold path's 4-row groups: a lane holds 4 columns of 4 rows
+  using T = Tile<RP, RN, 16>;   // the folds' 4-row groups: a lane holds 4 columns of 4 rows
   using Codes = RcCodes<RF>;
   constexpr int TB = tile_bytes<RF, RP, RN>();
   constexpr int RB = rc_row_bytes<RF, RN>();
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kRcThreads, 4) m2_rc_decode_kernel(const StepA
   const int st = rp.st, n = rp.n;
   const bool pre = rp.pre, post = rp.post, fold = pre || post;
   const int w0 = pre ? n : 0;
-  if (!early && !fold && warp < hc)
+  if (!early && !pre && warp < hc)
     load_batch<RF>(cq, a.rc_codes + ((size_t)rp.src * a.H + h0 + warp) * TB, a.rc_scales,
                    ((size_t)rp.src * a.H + h0 + warp) * RP, 0, lane);
 
@@ -319,7 +321,8 @@ __global__ void __launch_bounds__(kRcThreads, 4) m2_rc_decode_kernel(const StepA
     const Stage stg{sX + (size_t)jh * WM * kXRow, 0, kXRow, n, L};
     const float Ah = sA[jh];
     const float Dh = __ldg(a.D + h);
-    // output coefficients: lane i holds entry w0 + i
+    float *hs = ssc + jh * kHS;   // fold weights: [33, 65) the pre-fold, [65, 97) the window fold; decays 97, 98
+    // output coefficients (lane i: entry w0 + i) and the decay from the checkpoint
     const int len = n - w0 + 1;
     float coef, dec;
     {
@@ -329,96 +332,86 @@ __global__ void __launch_bounds__(kRcThreads, 4) m2_rc_decode_kernel(const StepA
       coef = lane < len ? expf(Ah * after) * v * sBC[w0 + lane] : 0.0f;
       dec = expf(Ah * total);
     }
-    if (!fold) {
-      // window terms of rows lane and lane + 32 (the codes' loads are in flight)
-      float ws[2] = {0.0f, 0.0f};
-      for (int i = 0; i < len; ++i) {
-        const float ci = __shfl_sync(kFull, coef, i);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) ws[q] = fmaf(ci, stg.x<Tin>(w0 + i, lane + 32 * q), ws[q]);
-      }
-      // tensor-core read of the copy, batch by batch (NVFP4: two batches of two
-      // 16-row m-tiles; FP8: four of one); the next batch, or the next head's
-      // first, is requested as soon as this one's codes are used
-#pragma unroll
-      for (int bi = 0; bi < Codes::kBatches; ++bi) {   // cq holds batch bi of this head
-        float hcv[Codes::kTiles];
-#pragma unroll
-        for (int k = 0; k < Codes::kTiles; ++k) hcv[k] = tile_hc<RF>(cq, k, cfrag, lane);
-        if (bi + 1 < Codes::kBatches) {
-          load_batch<RF>(cq, a.rc_codes + sbh * TB, a.rc_scales, sbh * RP, bi + 1, lane);
-        } else if (jh + kRcWarps < hc) {
-          const size_t nbh = sbh + kRcWarps;
-          load_batch<RF>(cq, a.rc_codes + nbh * TB, a.rc_scales, nbh * RP, 0, lane);
-        }
-        if constexpr (Codes::kTiles == 2) {   // rows 32 bi + lane: m-tile 2 bi + (lane >= 16)
-          const int row = 32 * bi + lane;
-          const float hcr = lane < 16 ? hcv[0] : hcv[1];
-          a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcr * cinv, ws[bi]));
-        } else {   // rows 16 bi + (lane & 15), written by lanes 0..15
-          const int row = 16 * bi + (lane & 15);
-          const float wsr = __shfl_sync(kFull, ws[bi >> 1], row & 31);
-          if (lane < 16)
-            a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcv[0] * cinv, wsr));
-        }
-      }
-    } else {
-      // ---- a fold this call: the general kernel's CUDA-core path, 4 rows at a
-      //      time, with this head's scalars in its slot of shared memory
-      float *hs = ssc + jh * kHS;
-      hs[lane] = coef;
-      if (lane == 0) hs[32] = dec;
-      for (int q = 0; q < 2; ++q) {
-        if (q == 0 ? !pre : !post) continue;
-        const int i0 = q == 0 ? 0 : w0, fl = q == 0 ? n : n - w0 + 1;
-        const float v = lane < fl ? sdt[jh * WM + i0 + lane] : 0.0f;
-        float after, total;
-        suffix_scan(v, lane, after, total);
-        hs[33 + q * 32 + lane] = expf(Ah * after) * v;
-        if (lane == 0) hs[97 + q] = expf(Ah * total);
-      }
+    // fold weights e^{A seg(i, last)} dt_i of a folded window [i0, i0 + ne) and its decay
+    auto fold_weights = [&](int q, int i0, int ne) {
+      const float v = lane < ne ? sdt[jh * WM + i0 + lane] : 0.0f;
+      float after, total;
+      suffix_scan(v, lane, after, total);
+      hs[33 + 32 * q + lane] = expf(Ah * after) * v;
+      if (lane == 0) hs[97 + q] = expf(Ah * total);
       __syncwarp();
-      const float *hcoef = hs, *hdec = hs + 32, *hfw = hs + 33, *hdecf = hs + 97;
-      const float *hc_src = a.hc + sbh * RP * RN;
-      float *hc_dst = a.hc + dbh * RP * RN;
-      uint8_t *rc_dst = a.rc_codes + dbh * TB;
-      const uint8_t *rc_src = a.rc_codes + sbh * TB;
-      const int c0 = lane * 4;
+    };
+    // fold entries [i0, i1) of the window into the fp32 checkpoint read at src,
+    // store it and quantise the new copy, 4 rows at a time (a lane: 4 columns
+    // of 4 rows)
+    const int c0 = lane * 4;
+    float *hc_dst = a.hc + dbh * RP * RN;
+    uint8_t *rc_dst = a.rc_codes + dbh * TB;
+    auto fold_rows = [&](const float *src, int i0, int i1, const float *fw, float fdec) {
 #pragma unroll 1
       for (int vw = 0; vw < RP / T::RPW; ++vw) {
         const int row0 = vw * T::RPW;
-        float4 v[T::NLD];
-        if (pre) {   // the token does not fit: fold the committed window, store, quantise the copy
-          float4 f[T::NLD];
+        float4 f[T::NLD];
 #pragma unroll
-          for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(hc_src + (size_t)(row0 + l) * RN + c0);
-          fold_tile<RP, RN, 16, Tin>(f, hfw, hdecf[0], 0, n, stg, sB, row0, c0);
+        for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(src + (size_t)(row0 + l) * RN + c0);
+        fold_tile<RP, RN, 16, Tin>(f, fw, fdec, i0, i1, stg, sB, row0, c0);
 #pragma unroll
-          for (int l = 0; l < T::NLD; ++l) {
-            const int row = row0 + l;
-            st_stream(hc_dst + (size_t)row * RN + c0, f[l]);
-            v[l] = quantize4<RF, T::LPR>(f[l], rc_dst + (size_t)row * RB, a.rc_scales, dbh * RP + row, RN, c0, lane);
-          }
-        } else {
-#pragma unroll
-          for (int l = 0; l < T::NLD; ++l)
-            v[l] = load_read_copy4<RF>(rc_src + (size_t)(row0 + l) * RB, a.rc_scales, sbh * RP + row0 + l, RN, c0);
-        }
-        outputs<RP, RN, 16, Tin, 1>(v, a, sC, hcoef, hdec, stg, b, h, n, w0, row0, lane, c0);
-        if (post) {   // the decode filled the window: fold it (after a pre-fold, from what that stored)
-          const float *fsrc = pre ? hc_dst : hc_src;
-          float4 f[T::NLD];
-#pragma unroll
-          for (int l = 0; l < T::NLD; ++l) f[l] = ld_stream(fsrc + (size_t)(row0 + l) * RN + c0);
-          fold_tile<RP, RN, 16, Tin>(f, hfw + 32, hdecf[1], w0, n + 1, stg, sB, row0, c0);
-#pragma unroll
-          for (int l = 0; l < T::NLD; ++l) {
-            const int row = row0 + l;
-            st_stream(hc_dst + (size_t)row * RN + c0, f[l]);
-            quantize4<RF, T::LPR>(f[l], rc_dst + (size_t)row * RB, a.rc_scales, dbh * RP + row, RN, c0, lane);
-          }
+        for (int l = 0; l < T::NLD; ++l) {
+          const int row = row0 + l;
+          st_stream(hc_dst + (size_t)row * RN + c0, f[l]);
+          quantize4<RF, T::LPR>(f[l], rc_dst + (size_t)row * RB, a.rc_scales, dbh * RP + row, RN, c0, lane);
         }
       }
+    };
+    size_t cbh = sbh;   // the copy the outputs read
+    if (pre) {
+      // the token does not fit: fold the committed window first; the outputs
+      // then read the copy this writes (the warp's own stores: fence, then sync)
+      fold_weights(0, 0, n);
+      fold_rows(a.hc + sbh * RP * RN, 0, n, hs + 33, hs[97]);
+      __threadfence_block();
+      __syncwarp();
+      cbh = dbh;
+      load_batch<RF>(cq, a.rc_codes + cbh * TB, a.rc_scales, cbh * RP, 0, lane);
+    } else if (post && jh != warp) {   // after a fold the next head's codes are requested at its start
+      load_batch<RF>(cq, a.rc_codes + cbh * TB, a.rc_scales, cbh * RP, 0, lane);
+    }
+    // ---- outputs: window terms of rows lane and lane + 32 (while the codes'
+    //      loads are in flight), then the tensor-core read of the copy, batch by
+    //      batch (NVFP4: two batches of two 16-row m-tiles; FP8: four of one);
+    //      the next batch, or without a fold the next head's first, is requested
+    //      as soon as this one's codes are used
+    float ws[2] = {0.0f, 0.0f};
+    for (int i = 0; i < len; ++i) {
+      const float ci = __shfl_sync(kFull, coef, i);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) ws[q] = fmaf(ci, stg.x<Tin>(w0 + i, lane + 32 * q), ws[q]);
+    }
+#pragma unroll
+    for (int bi = 0; bi < Codes::kBatches; ++bi) {   // cq holds batch bi of this head's copy
+      float hcv[Codes::kTiles];
+#pragma unroll
+      for (int k = 0; k < Codes::kTiles; ++k) hcv[k] = tile_hc<RF>(cq, k, cfrag, lane);
+      if (bi + 1 < Codes::kBatches) {
+        load_batch<RF>(cq, a.rc_codes + cbh * TB, a.rc_scales, cbh * RP, bi + 1, lane);
+      } else if (!fold && jh + kRcWarps < hc) {
+        const size_t nbh = sbh + kRcWarps;
+        load_batch<RF>(cq, a.rc_codes + nbh * TB, a.rc_scales, nbh * RP, 0, lane);
+      }
+      if constexpr (Codes::kTiles == 2) {   // rows 32 bi + lane: m-tile 2 bi + (lane >= 16)
+        const int row = 32 * bi + lane;
+        const float hcr = lane < 16 ? hcv[0] : hcv[1];
+        a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcr * cinv, ws[bi]));
+      } else {   // rows 16 bi + (lane & 15), written by lanes 0..15
+        const int row = 16 * bi + (lane & 15);
+        const float wsr = __shfl_sync(kFull, ws[bi >> 1], row & 31);
+        if (lane < 16)
+          a.out[((size_t)b * a.H + h) * RP + row] = fmaf(Dh, stg.x<Tin>(n, row), fmaf(dec, hcv[0] * cinv, wsr));
+      }
+    }
+    if (post) {   // the window is full: fold it (after a pre-fold, on top of what that stored)
+      fold_weights(1, w0, n - w0 + 1);
+      fold_rows(pre ? hc_dst : a.hc + sbh * RP * RN, w0, n + 1, hs + 65, hs[98]);
     }
   }
 }
