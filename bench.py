@@ -182,6 +182,7 @@ class Mamba2Work:
     name = "mamba2"
     keys = ("x", "B", "C", "dt")
     kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/mamba2.cu",
+                    "hybrid_ssm_decode_replayssm_b200/csrc/m2_common.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/umma.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
                     "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
@@ -213,8 +214,17 @@ class Mamba2Work:
     def drafts(self, rnd, k):
         return [t.to(self.dev) for t in (si.mamba2_drafts(self.shape, rnd, k, self.seed)[n] for n in self.keys)]
 
+    rc_kernel_files = ["hybrid_ssm_decode_replayssm_b200/csrc/m2_rc_decode.cu",
+                       "hybrid_ssm_decode_replayssm_b200/csrc/m2_common.cuh",
+                       "hybrid_ssm_decode_replayssm_b200/csrc/rssm_device.cuh",
+                       "hybrid_ssm_decode_replayssm_b200/csrc/rssm_internal.h"]
+
     def bytes_per_call(self, pos):
-        """Algorithmic bytes of the decode call at window position pos (1..L)."""
+        """Algorithmic bytes of the decode call at window position pos (1..L):
+        the state read (fp32 checkpoint, or the read copy's codes and scales),
+        token inputs, the ring append, the window entries before it, the output;
+        at pos = L the fold writes the checkpoint (a read-copy layer also reads
+        the fp32 checkpoint then, and writes the new copy)."""
         s = self.shape
         B, H, P, N, G, L = s.batch, s.nheads, s.headdim, s.dstate, s.ngroups, s.window
         e = 2
@@ -222,7 +232,12 @@ class Mamba2Work:
         inp = B * H * P * e + 2 * B * G * N * e + B * H * e
         entry = B * H * P * e + B * G * N * e + B * H * 4
         out = B * H * P * 4
-        return ck + inp + entry + (pos - 1) * entry + out + (ck if pos == L else 0)
+        if self.read_fmt == 0:
+            read, fold = ck, ck
+        else:
+            rc = B * H * P * N + B * H * P * 4 if self.read_fmt == 1 else B * H * P * N // 2 + B * H * P * N // 16
+            read, fold = rc, 2 * ck + rc
+        return read + inp + entry + (pos - 1) * entry + out + (fold if pos == L else 0)
 
     def conventional_bytes(self):
         s = self.shape
@@ -661,6 +676,7 @@ def _window_layer(base, L, fmt):
     work.shape = base.shape.with_(window=L, max_draft=min(base.shape.max_draft, L))
     work.desc = copy.copy(base.desc)
     work.desc.window, work.desc.max_draft, work.desc.read_fmt = L, min(base.shape.max_draft, L), fmt
+    work.read_fmt = fmt
     return work
 
 
@@ -671,7 +687,7 @@ def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6, err_calls=64):
     checkpoint (which the parity tests hold to the fp64 oracle at ~1e-6): per
     call |y_copy - y_fp32| / rms(y_fp32), max and rms over `err_calls` calls."""
     from hybrid_ssm_decode_replayssm_b200 import rssm
-    res, err = {}, {}
+    res, err, gbs = {}, {}, {}
     fmts = (("fp32", rssm.RSSM_READ_FP32), ("fp8_e4m3_row", rssm.RSSM_READ_FP8_E4M3_ROW),
             ("nvfp4", rssm.RSSM_READ_NVFP4))
     for name, fmt in fmts:
@@ -682,6 +698,9 @@ def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6, err_calls=64):
             n_windows = max(2, (steps * 16) // L)
             el = time_plain_decode(work, layer, n_windows, 2, L)
             row[f"L{L}"] = round(work.shape.batch * L * n_windows / el, 1)
+            if work.name == "mamba2":   # HBM bytes per second (algorithmic bytes of the window's calls)
+                gbs.setdefault(name, {})[f"L{L}"] = round(
+                    sum(work.bytes_per_call(p) for p in range(1, L + 1)) * n_windows / el / 1e9, 1)
             del layer
             torch.cuda.empty_cache()
         res[name] = row
@@ -705,6 +724,8 @@ def read_copy_leg(base, windows=(1, 4, 8, 16, 32), steps=6, err_calls=64):
             torch.cuda.empty_cache()
         err[name] = row
     res["error_vs_fp32_reads"] = err
+    if gbs:
+        res["hbm_gbs"] = gbs
     return res
 
 
@@ -800,6 +821,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch (profiling captures only; the metric is quoted at 256)")
+    ap.add_argument("--read-fmt", default="fp32", choices=["fp32", "fp8", "nvfp4"],
+                    help="read format of the timed layer (profiling captures only; the metric is quoted on fp32 reads)")
     ap.add_argument("--legs", default="replay,conventional,e2e,gdn,kda,speculative,read_copy,quantized_state,graph,branch",
                     help="comma list of timed legs (profiling captures run 'replay' alone)")
     args = ap.parse_args()
@@ -821,7 +844,7 @@ def main():
         torch.cuda.set_device(dev)
     seed = args.seed + rank
     legs = set(args.legs.split(","))
-    work = WORKLOADS[args.layer](dev, seed, args.batch)
+    work = WORKLOADS[args.layer](dev, seed, args.batch, read_fmt={"fp32": 0, "fp8": 1, "nvfp4": 2}[args.read_fmt])
     L = work.shape.window
     tokens_per_step = work.tokens_per_call * L
     cfg = {"workload": work.workload, "global_batch": work.shape.batch * world,
@@ -854,7 +877,10 @@ def main():
     kern_time = sum(per)
     peak, peak_kind = measured_peak()
     achieved = alg_bytes / kern_time / 1e9
-    traffic = ncu_traffic(f"{work.name}_decode", work.kernel_files)
+    if work.read_fmt == 0:
+        traffic = ncu_traffic(f"{work.name}_decode", work.kernel_files)
+    else:
+        traffic = ncu_traffic(f"{work.name}_rc{work.read_fmt}_decode", getattr(work, "rc_kernel_files", work.kernel_files))
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),

@@ -220,6 +220,8 @@ int rssm_set_wait_limit(rssm_handle *h, long long cycles);
  * after the handle's wait limit, sets RSSM_STATUS_TIMEOUT and the CTA ends
  * early, exactly as a copy that never lands would make it.  Nothing faults or
  * hangs; the launch's results are unspecified (call rssm_reset afterwards).
+ * Decodes of Mamba-2 read-copy layers with bf16 inputs (headdim 64, dstate
+ * 128) run a kernel without waits: such a launch just clears the armed test.
  * KDA: only the decode serving kernel (bf16 inputs) waits, so only a decode of
  * such a handle takes the path (a verify or flush launch just clears the armed
  * test); a KDA handle with fp32 inputs gives RSSM_ERR_UNSUPPORTED. */
