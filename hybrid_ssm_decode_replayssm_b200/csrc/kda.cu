@@ -80,8 +80,9 @@ __device__ __forceinline__ void kda_decays(const float *aw, float *dec, float *e
   }
 }
 
-template <typename Tin>
+template <typename Tin, int RF>
 __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepArgs a) {
+  constexpr int RB = RF == RSSM_READ_NVFP4 ? KD / 2 : KD;   // bytes of a read-copy row
   extern __shared__ __align__(16) float sm[];
   const int bh = blockIdx.x, b = bh / a.H, h = bh - b * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -99,8 +100,18 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   const int src_slot = a.slot ? a.slot[b] : b;
   const float *src = a.hc + ((size_t)src_slot * a.H + h) * KD * KD;
   float4 S[kRowsPerWarp];
+  auto load_fp32 = [&](const float *from) {
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) S[i] = ld_stream(src + (size_t)(row0 + i) * KD + c0);
+    for (int i = 0; i < kRowsPerWarp; ++i) S[i] = ld_stream(from + (size_t)(row0 + i) * KD + c0);
+  };
+  if constexpr (RF == RSSM_READ_FP32) {
+    load_fp32(src);
+  } else {   // a read-copy layer's reads see the copy; a fold reloads the fp32 rows
+    const size_t rbase = ((size_t)src_slot * a.H + h) * KD;
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i)
+      S[i] = load_read_copy4<RF>(a.rc_codes + (rbase + row0 + i) * RB, a.rc_scales, rbase + row0 + i, KD, c0);
+  }
   // and the first new token's inputs (thread c < KD: channel / value row c)
   Tin kr{}, vr{}, qr{};
   float ar = 1.0f;
@@ -159,6 +170,59 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
 
   float *dst = a.hc + ((size_t)rp.dst * a.H + h) * KD * KD;   // where a fold writes
 
+  // Read-copy layers: the w rows cached while decoding were solved against the
+  // copy, so a fold first solves its entries 0..tl again against the fp32 tile
+  // in S (the same forward substitution; entry t in ring slot (st_e + t) % cap),
+  // leaving dec / eG of t = tl for the fold.  The cached rows are not rewritten:
+  // the fold empties the window.
+  auto resolve = [&](int tl, int st_e) {
+    for (int t = 0; t <= tl; ++t) {
+      const size_t slot = (size_t)((st_e + t) % cap);
+      kda_decays(gw, dec, eG, t);
+      __syncthreads();
+      for (int s2 = warp; s2 < t; s2 += kKdaThreads / 32) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < KD / 32; ++jj) {
+          const int c = lane + 32 * jj;
+          acc = fmaf(kw[s2 * KD + c] * dec[s2 * KD + c], kw[t * KD + c], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) Adot[s2] = acc;
+      }
+      {   // u = S (e^{G_t} . k_t)
+        const float4 e = *reinterpret_cast<const float4 *>(eG + c0);
+        const float4 kk = *reinterpret_cast<const float4 *>(kw + t * KD + c0);
+        const float4 gk = make_float4(e.x * kk.x, e.y * kk.y, e.z * kk.z, e.w * kk.w);
+        float p[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) p[i] = S[i].x * gk.x + S[i].y * gk.y + S[i].z * gk.z + S[i].w * gk.w;
+        tr_sum<kRowsPerWarp, 16>(p, lane);   // lanes 2j, 2j + 1 hold the sum of row tr_base
+        if ((lane & 1) == 0) uu[row0 + tr_base<kRowsPerWarp, 16>(lane)] = p[0];
+      }
+      __syncthreads();
+      if (tid < KD) {
+        float r = to_f32<Tin>(vring[slot * KD + tid]) - uu[tid];
+        for (int s2 = 0; s2 < t; ++s2) r = fmaf(-Adot[s2], ww[s2 * KD + tid], r);
+        ww[t * KD + tid] = bring[slot] * r;
+      }
+      __syncthreads();
+    }
+  };
+  // Store the folded fp32 rows; a read-copy layer also quantises them into its
+  // copy and reads the copy back into S (the reads that follow see the new copy).
+  auto store_fold = [&]() {
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
+    if constexpr (RF != RSSM_READ_FP32) {
+      const size_t dbase = ((size_t)rp.dst * a.H + h) * KD;
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i)
+        S[i] = quantize4<RF, 32>(S[i], a.rc_codes + (dbase + row0 + i) * RB, a.rc_scales, dbase + row0 + i, KD, c0,
+                                 lane);
+    }
+  };
+
   // committed window rows into shared memory
   for (int idx = tid; idx < n * KD; idx += kKdaThreads) {
     const int e = idx / KD, c = idx - e * KD;
@@ -170,12 +234,19 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   __syncthreads();
 
   if (pre) {   // the committed window is folded first (flush, or a token that does not fit)
-    kda_decays(gw, dec, eG, n - 1);
-    __syncthreads();
-    kda_fold(S, eG, kw, dec, ww, n - 1, row0, c0);
-    if (!post && m == 0) {
+    if constexpr (RF == RSSM_READ_FP32) {
+      kda_decays(gw, dec, eG, n - 1);
+      __syncthreads();
+      kda_fold(S, eG, kw, dec, ww, n - 1, row0, c0);
+      if (!post && m == 0) {
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
+        for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
+      }
+    } else {
+      load_fp32(src);
+      resolve(n - 1, st);
+      kda_fold(S, eG, kw, dec, ww, n - 1, row0, c0);
+      store_fold();
     }
     __syncthreads();   // the window arrays are reused below
   }
@@ -257,10 +328,17 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_replay_kernel(const StepAr
   }
   if (m >= 1) {
     if (post) {   // the decode filled the window: fold all of it
-      kda_fold(S, eG, kw, dec, ww, n, row0, c0);
+      if constexpr (RF == RSSM_READ_FP32) {
+        kda_fold(S, eG, kw, dec, ww, n, row0, c0);
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
-    } else if (pre) {
+        for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
+      } else {   // from the fp32 rows (those a pre-fold of this call stored, if any)
+        load_fp32(pre ? dst : src);
+        resolve(n, st_new);
+        kda_fold(S, eG, kw, dec, ww, n, row0, c0);
+        store_fold();
+      }
+    } else if (pre && RF == RSSM_READ_FP32) {   // (a read-copy layer stored its pre-fold already)
 #pragma unroll
       for (int i = 0; i < kRowsPerWarp; ++i) st_stream(dst + (size_t)(row0 + i) * KD + c0, S[i]);
     }
@@ -318,9 +396,9 @@ __global__ void __launch_bounds__(kKdaThreads, 2) kda_conv_kernel(const ConvArgs
   if ((lane & 1) == 0) a.out[(size_t)bh * KD + row0 + tr_base<kRowsPerWarp, 16>(lane)] = a.out_scale * p[0];
 }
 
-template <typename Tin>
+template <typename Tin, int RF>
 cudaError_t launch_kda_step(const StepArgs &a, cudaStream_t s) {
-  auto kern = kda_replay_kernel<Tin>;
+  auto kern = kda_replay_kernel<Tin, RF>;
   const KdaSmem y{a.L + (a.m > 1 ? a.m : 1)};   // the window and the new tokens
   const size_t smem = y.floats() * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -329,13 +407,22 @@ cudaError_t launch_kda_step(const StepArgs &a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <typename Tin>
+cudaError_t dispatch_rf(const StepArgs &a, int read_fmt, cudaStream_t s) {
+  switch (read_fmt) {
+    case RSSM_READ_FP32: return launch_kda_step<Tin, RSSM_READ_FP32>(a, s);
+    case RSSM_READ_FP8_E4M3_ROW: return launch_kda_step<Tin, RSSM_READ_FP8_E4M3_ROW>(a, s);
+    default: return launch_kda_step<Tin, RSSM_READ_NVFP4>(a, s);
+  }
+}
+
 }  // namespace
 
 bool kda_supported(int R, int C) { return R == KD && C == KD; }
 
-cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s) {
+cudaError_t kda_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s) {
   if (kda_decode_fast_path(a, in_dtype)) return kda_decode_step(a, s);
-  return in_dtype == RSSM_BF16 ? launch_kda_step<__nv_bfloat16>(a, s) : launch_kda_step<float>(a, s);
+  return in_dtype == RSSM_BF16 ? dispatch_rf<__nv_bfloat16>(a, read_fmt, s) : dispatch_rf<float>(a, read_fmt, s);
 }
 
 cudaError_t kda_conventional(const ConvArgs &a, int in_dtype, cudaStream_t s) {

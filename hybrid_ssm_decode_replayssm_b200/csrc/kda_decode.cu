@@ -665,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_decode_kernel(const StepArgs 
 
 bool kda_decode_fast_path(const StepArgs &a, int in_dtype) {
   return a.mode == kDecode && a.m == 1 && in_dtype == RSSM_BF16 && a.R == DV && a.C == DK && a.L <= kW &&
-         a.fold_scratch != nullptr;
+         a.fold_scratch != nullptr && a.rc_codes == nullptr;
 }
 
 static int heads_per_item(int H) {
@@ -675,7 +675,8 @@ static int heads_per_item(int H) {
 }
 
 size_t kda_fold_scratch_bytes(const rssm_layer_desc &d) {
-  if (d.in_dtype != RSSM_BF16 || d.headdim != DV || d.dstate != DK || d.window > kW) return 0;
+  if (d.in_dtype != RSSM_BF16 || d.read_fmt != RSSM_READ_FP32 || d.headdim != DV || d.dstate != DK || d.window > kW)
+    return 0;
   const int hc = heads_per_item(d.nheads);
   const size_t items = (size_t)d.batch * (d.nheads / hc);
   const size_t ctas = items < (size_t)kScratchCtas ? items : (size_t)kScratchCtas;

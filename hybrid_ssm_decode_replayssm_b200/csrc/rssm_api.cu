@@ -74,8 +74,6 @@ int validate_desc(const rssm_layer_desc *d) {
   if (!sup)
     return fail(RSSM_ERR_UNSUPPORTED, "no kernel for %s headdim=%d dstate=%d in this build",
                 d->kind == RSSM_MAMBA2 ? "Mamba-2" : d->kind == RSSM_GDN ? "GDN" : "KDA", d->headdim, d->dstate);
-  if (d->kind == RSSM_KDA && d->read_fmt != RSSM_READ_FP32)
-    return fail(RSSM_ERR_UNSUPPORTED, "KDA layers read the fp32 checkpoint (no read copy in this build)");
   return RSSM_OK;
 }
 
@@ -215,7 +213,7 @@ cudaError_t replay_launch(const rssm_handle *h, const rssm::StepArgs &a, cudaStr
   switch (h->d.kind) {
     case RSSM_MAMBA2: return rssm::mamba2_step(a, h->d.in_dtype, h->d.read_fmt, s);
     case RSSM_GDN: return rssm::gdn_step(a, h->d.in_dtype, h->d.read_fmt, s);
-    default: return rssm::kda_step(a, h->d.in_dtype, s);
+    default: return rssm::kda_step(a, h->d.in_dtype, h->d.read_fmt, s);
   }
 }
 
@@ -405,6 +403,8 @@ int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev, c
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.read_fmt == RSSM_READ_FP32)
     return fail(RSSM_ERR_STATE, "the layer has no low-precision format (read_fmt is RSSM_READ_FP32)");
+  if (h->d.kind == RSSM_KDA)
+    return fail(RSSM_ERR_UNSUPPORTED, "no stored low-precision state baseline for KDA layers");
   if (!codes_in_dev || !scales_in_dev || !codes_out_dev || !scales_out_dev)
     return fail(RSSM_ERR_INVALID_ARG, "state code and scale pointers must not be NULL");
   if (!aligned(codes_in_dev, 16) || !aligned(codes_out_dev, 16))

@@ -6,8 +6,9 @@
 namespace rssm {
 
 bool kda_supported(int R, int C);
-// decode (m = 1), verify (m = k drafts) and flush (m = 0)
-cudaError_t kda_step(const StepArgs &a, int in_dtype, cudaStream_t s);
+// decode (m = 1), verify (m = k drafts) and flush (m = 0); read_fmt: the
+// layer's read copy (RSSM_READ_FP32: none)
+cudaError_t kda_step(const StepArgs &a, int in_dtype, int read_fmt, cudaStream_t s);
 // The decode serving path (one token, bf16 inputs): its own persistent kernel
 // with prologue warps and tensor-core folds (kda_decode.cu).
 bool kda_decode_fast_path(const StepArgs &a, int in_dtype);

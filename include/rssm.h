@@ -98,8 +98,9 @@ enum {
  *            mapping keys to values; ngroups is ignored.
  *   KDA:     as GDN, with one gate per key channel (Kimi Delta Attention,
  *            named by [teaser]; read as S <- S Diag(alpha) (I - beta k k^T)
- *            + beta v k^T, o = out_scale S q): replay decode and flush on the
- *            fp32 checkpoint; no read copy, no verify in this build.
+ *            + beta v k^T, o = out_scale S q): replay decode, verify and flush;
+ *            with a read copy the reads see the copy and every fold solves
+ *            the window again from the fp32 checkpoint (as GDN).
  * A "row" of the state is its last dimension: the contraction vector of one
  * output element (h[b,h,p,:] or S[b,h,i,:]).
  * Supported by this build: Mamba-2 headdim 64 with dstate 64 or 128;
@@ -107,7 +108,7 @@ enum {
  * max_draft <= window.
  */
 typedef struct {
-  int kind;        /* RSSM_MAMBA2 | RSSM_GDN                                  */
+  int kind;        /* RSSM_MAMBA2 | RSSM_GDN | RSSM_KDA                       */
   int batch;       /* sequences B                                             */
   int nheads;      /* H                                                       */
   int ngroups;     /* Mamba-2 G (nheads % ngroups == 0); GDN: ignored         */
@@ -311,7 +312,8 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev,
  * handle's shape, formats and parameters; its checkpoint, read copy and
  * window are untouched.
  * Errors: RSSM_ERR_STATE if read_fmt is RSSM_READ_FP32; RSSM_ERR_INVALID_ARG
- * for NULL or misaligned pointers (codes 16-byte, FP8 scales 4-byte aligned).
+ * for NULL or misaligned pointers (codes 16-byte, FP8 scales 4-byte aligned);
+ * RSSM_ERR_UNSUPPORTED for KDA layers (Mamba-2 and GDN only).
  */
 int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev,
                                      const void *scales_in_dev,

@@ -35,7 +35,10 @@ int main(void) {
   d.kind = RSSM_KDA;
   d.headdim = d.dstate = 128;
   d.read_fmt = RSSM_READ_NVFP4;
-  if (rssm_workspace_size(&d, &ck, &buf, &rc, &meta, &lay) != RSSM_ERR_UNSUPPORTED) return 6;
+  if (rssm_workspace_size(&d, &ck, &buf, &rc, &meta, &lay) != RSSM_OK || rc == 0) return 6;
+  d.headdim = 64;
+  if (rssm_workspace_size(&d, &ck, &buf, &rc, &meta, &lay) != RSSM_ERR_UNSUPPORTED) return 11;
+  d.headdim = 128;
   if (rssm_branch(NULL, NULL, NULL) != RSSM_ERR_INVALID_ARG) return 7;
   if (rssm_decode_step(NULL, NULL, NULL, NULL) != RSSM_ERR_INVALID_ARG) return 8;
   size_t n = 0;

@@ -76,10 +76,11 @@ def gdn_layer(shape: si.GDNLayer, read_fmt=rssm.RSSM_READ_FP32, auto_flush=True,
 KDA_KEYS = ("q", "k", "v", "alpha", "beta")
 
 
-def kda_layer(shape, auto_flush=True, seed=0, out_scale=1.0, branching=False, max_draft=0):
+def kda_layer(shape, auto_flush=True, seed=0, out_scale=1.0, branching=False, max_draft=0,
+              read_fmt=rssm.RSSM_READ_FP32):
     S0 = si.kda_checkpoint(shape, seed)
     desc = rssm.make_desc(rssm.RSSM_KDA, shape.batch, shape.nheads, shape.dv, shape.dk, window=shape.window,
                           max_draft=max_draft, in_dtype=rssm.RSSM_BF16 if shape.dtype == "bf16" else rssm.RSSM_F32,
-                          auto_flush=auto_flush, out_scale=out_scale, branching=branching)
+                          auto_flush=auto_flush, out_scale=out_scale, branching=branching, read_fmt=read_fmt)
     layer = rssm.ReplayLayer(desc, _ckpt(S0, branching))
     return layer, S0

@@ -207,7 +207,10 @@ def test_kda_descriptor_and_layout():
     assert lay.buf_off[1] >= B * H * cap * d * 2                       # k ring (bf16)
     assert lay.buf_off[3] - lay.buf_off[2] >= B * H * cap * d * 4      # per-channel log gates (fp32)
     assert buf >= lay.buf_off[4] + B * H * cap * d * 4                 # w rows (fp32)
-    assert _sizes(_desc(**dict(base, read_fmt=rssm.RSSM_READ_NVFP4)))[0] == rssm.RSSM_ERR_UNSUPPORTED
+    code, (_, _, rc4, _), _ = _sizes(_desc(**dict(base, read_fmt=rssm.RSSM_READ_NVFP4)))
+    assert code == rssm.RSSM_OK and rc4 == 2 * 4 * 128 * 64 + 2 * 4 * 128 * 8   # codes + E4M3 scales
+    code, (_, _, rc8, _), _ = _sizes(_desc(**dict(base, read_fmt=rssm.RSSM_READ_FP8_E4M3_ROW)))
+    assert code == rssm.RSSM_OK and rc8 == 2 * 4 * 128 * 128 + 2 * 4 * 128 * 4    # codes + fp32 row scales
     assert _sizes(_desc(**dict(base, headdim=64)))[0] == rssm.RSSM_ERR_UNSUPPORTED
     L = rssm.lib()
     fake = 1 << 20

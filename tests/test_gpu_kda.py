@@ -12,7 +12,11 @@ window when it fills, and must give the recurrence's outputs and states:
 * explicit masked flush, restore to a position, and branching (rows sharing
   checkpoint slots) against the oracle's window rules;
 * speculative verify of k drafts with rollback to the accepted prefix against
-  the oracle's round (oracle.speculative.kda_round), and its refusals.
+  the oracle's round (oracle.speculative.kda_round), and its refusals;
+* FP8-row / NVFP4 read copies: the copy is always the oracle codec's quantisation
+  of the fp32 checkpoint (code for code), the outputs are the recurrence from
+  the copy's values, and every fold solves the window again from the fp32
+  checkpoint, which tracks the exact state.
 """
 import numpy as np
 import pytest
@@ -23,6 +27,7 @@ from gpu_common import DEV, KDA_KEYS, assert_close, dev_inputs, kda_layer, to64,
 from hybrid_ssm_decode_replayssm_b200 import rssm
 from oracle import bookkeeping as obk
 from oracle import branch as ob
+from oracle import codecs as oc
 from oracle import kda as ok
 from oracle import speculative as osp
 
@@ -165,3 +170,89 @@ def test_verify_refusals():
     assert layer.get_status(clear=True) == rssm.RSSM_STATUS_CAPACITY
     assert _bk(layer) == before
     assert_close(layer.ckpt.cpu(), to64(S0), 0.0, "checkpoint untouched")
+
+
+FMTS = [rssm.RSSM_READ_FP8_E4M3_ROW, rssm.RSSM_READ_NVFP4]
+
+
+def _read_view(layer, fmt, what):
+    """The layer's read copy checked code for code against the oracle codec applied
+    to its fp32 checkpoint; returns the copy's values (fp64), what the reads see."""
+    codes, scales = (t.cpu().numpy() for t in layer.read_copy_views())
+    if fmt == rssm.RSSM_READ_NVFP4:
+        codes = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(codes.shape[:-1] + (-1,))
+        want_codes, want_scales = oc.nvfp4_quantize(layer.ckpt.cpu().numpy())
+        deq = oc.nvfp4_dequantize(want_codes, want_scales)
+        np.testing.assert_array_equal(scales, want_scales, err_msg=what)
+    else:
+        want_codes, want_scales = oc.fp8_row_quantize(layer.ckpt.cpu().numpy())
+        deq = oc.fp8_row_dequantize(want_codes, want_scales)
+        np.testing.assert_array_equal(scales.view(np.uint32), want_scales.view(np.uint32), err_msg=what)
+    np.testing.assert_array_equal(codes, want_codes, err_msg=what)
+    return np.asarray(deq, dtype=np.float64)
+
+
+def _rows(mask):
+    return np.asarray(mask, dtype=bool)[:, None, None, None]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_read_copy_reads_and_fp32_folds(fmt):
+    """Decodes and verify rounds (seeded acceptance) on a layer with a read copy,
+    rows folding at different calls (window full, or drafts that do not fit), then
+    a flush.  The reads see the copy: every output equals the recurrence started
+    from the copy's values R (after a pre-fold, from the new copy).  The copy is
+    the quantised fp32 checkpoint at all times, and after each fold that
+    checkpoint equals the exact state S of the committed tokens."""
+    B, L, k = 3, 6, 3
+    shape = si.KDALayer(batch=B, nheads=4, dk=128, dv=128, window=L, dtype="bf16", state_std=0.05)
+    layer, S0 = kda_layer(shape, max_draft=k, read_fmt=fmt)
+    S = to64(S0)
+    R = _read_view(layer, fmt, "copy at creation")
+    book = obk.WindowBook(B, L, int(layer.layout.cap))
+    o = torch.empty(B, 4, 128, device=DEV)
+    ov = torch.empty(B, k, 4, 128, device=DEV)
+    ops = "ddvdvddvvdddvdvd"
+    for i, op in enumerate(ops):
+        if op == "d":
+            tok = si.kda_tokens(shape, 100 + i, seed=7)
+            plan = book.decode()
+            layer.decode_step(dev_inputs(tok, KDA_KEYS), o)
+            pre = [p[1] for p in plan]
+            post = [p[3] for p in plan]
+            C = _read_view(layer, fmt, f"copy after call {i}")
+            start = np.where(_rows(pre), C, R)
+            R_next, y = _step(start, tok64(tok))
+            assert_close(o.cpu(), y, TOL["bf16"], f"{fmt} decode {i}: outputs from the copy")
+            S_next, _ = _step(S, tok64(tok))
+            for b in range(B):
+                if post[b]:
+                    assert_close(layer.ckpt[b].cpu(), S_next[b], TOL["f32"], f"decode {i} row {b}: folded checkpoint")
+                elif pre[b]:
+                    assert_close(layer.ckpt[b].cpu(), S[b], TOL["f32"], f"decode {i} row {b}: pre-folded checkpoint")
+            R = np.where(_rows(post), C, R_next)
+            S = S_next
+        else:
+            drafts = si.kda_drafts(shape, i, k, seed=7)
+            acc = si.accept_counts(B, i, k, seed=7)
+            plan = book.verify(k)
+            layer.verify(k, dev_inputs(drafts, KDA_KEYS), ov)
+            pre = [p[1] for p in plan]
+            C = _read_view(layer, fmt, f"copy after call {i}")
+            want, R_next = osp.kda_round(np.where(_rows(pre), C, R), tok64(drafts), acc.numpy())
+            assert_close(ov.cpu(), want, TOL["bf16"], f"{fmt} verify {i}: outputs from the copy")
+            for b in range(B):
+                if pre[b]:
+                    assert_close(layer.ckpt[b].cpu(), S[b], TOL["f32"], f"verify {i} row {b}: pre-folded checkpoint")
+            _, S = osp.kda_round(S, tok64(drafts), acc.numpy())
+            n_reject = (k - acc).to(torch.int32)
+            layer.rollback(n_reject.to(DEV))
+            book.rollback(n_reject.tolist())
+            R = R_next
+        assert _bk(layer) == [list(x) for x in book.snapshot()], f"pointers after call {i}"
+    assert sum(book.flushes) >= 2 * B, "the sequence should fold every row more than once"
+    layer.flush()
+    book.flush()
+    assert_close(layer.ckpt.cpu(), S, TOL["f32"], "checkpoint after the final flush")
+    _read_view(layer, fmt, "copy after the final flush")
+    assert layer.get_status() == 0
