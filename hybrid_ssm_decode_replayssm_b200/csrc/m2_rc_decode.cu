@@ -17,8 +17,11 @@
 // heads), several CTAs resident per SM, and each warp loads its own head's
 // codes and scales straight into registers (requested before the CTA's
 // shared prologue so that their latency hides behind it) and multiplies them
-// with C on the tensor cores (mma.sync m16n8k16, f16 in, fp32 out; exact, see
-// m2_common.cuh).  The CTA's prologue stages the window: B rows (fp32), C,
+// with C on the tensor cores (mma.sync m16n8k16, f16 in, fp32 out).  The
+// products are exact: a dequantised code is exact in f16 (an E2M1 value times
+// an E4M3 block scale has at most 6 significant bits and lies in [2^-10, 2688];
+// an E4M3 code is exact, its fp32 row scale is applied to the sum), and C is
+// scaled by a power of two into [2^14, 2^15) before rounding to f16.  The CTA's prologue stages the window: B rows (fp32), C,
 // the dt windows, B.C, the window scalars and every head's x rows, with the
 // ring appends.  A row that folds this call does so on the CUDA cores, 4 state
 // rows at a time (fp32 read, rank-l update, fp32 store, new copy); its outputs
