@@ -212,7 +212,8 @@ def test_read_copy_reads_and_fp32_folds(fmt):
     book = obk.WindowBook(B, L, int(layer.layout.cap))
     o = torch.empty(B, 4, 128, device=DEV)
     ov = torch.empty(B, k, 4, 128, device=DEV)
-    ops = "ddvdvddvvdddvdvd"
+    ops = "ddvdvddvvdddvdvddvd"
+    pre_seen = post_seen = 0
     for i, op in enumerate(ops):
         if op == "d":
             tok = si.kda_tokens(shape, 100 + i, seed=7)
@@ -230,11 +231,13 @@ def test_read_copy_reads_and_fp32_folds(fmt):
                     assert_close(layer.ckpt[b].cpu(), S_next[b], TOL["f32"], f"decode {i} row {b}: folded checkpoint")
                 elif pre[b]:
                     assert_close(layer.ckpt[b].cpu(), S[b], TOL["f32"], f"decode {i} row {b}: pre-folded checkpoint")
+            pre_seen += sum(pre)
+            post_seen += sum(post)
             R = np.where(_rows(post), C, R_next)
             S = S_next
         else:
             drafts = si.kda_drafts(shape, i, k, seed=7)
-            acc = si.accept_counts(B, i, k, seed=7)
+            acc = si.accept_counts(B, i, k, seed=5)   # (this seed leaves some rows full before a decode)
             plan = book.verify(k)
             layer.verify(k, dev_inputs(drafts, KDA_KEYS), ov)
             pre = [p[1] for p in plan]
@@ -250,7 +253,7 @@ def test_read_copy_reads_and_fp32_folds(fmt):
             book.rollback(n_reject.tolist())
             R = R_next
         assert _bk(layer) == [list(x) for x in book.snapshot()], f"pointers after call {i}"
-    assert sum(book.flushes) >= 2 * B, "the sequence should fold every row more than once"
+    assert pre_seen > 0 and post_seen > 0, (pre_seen, post_seen)
     layer.flush()
     book.flush()
     assert_close(layer.ckpt.cpu(), S, TOL["f32"], "checkpoint after the final flush")

@@ -316,3 +316,84 @@ def test_many_items_per_cta(fmt):
     assert_close(layer.ckpt.cpu(), h, TOL["bf16"], "checkpoint")
     assert _bk(layer) == [list(x) for x in book.snapshot()]
     assert layer.get_status() == 0
+
+
+def _read_view(layer, fmt, what):
+    """The layer's read copy checked code for code against the oracle codec applied
+    to its fp32 checkpoint; returns the copy's values (fp64), what the reads see."""
+    codes, scales = (t.cpu().numpy() for t in layer.read_copy_views())
+    if fmt == rssm.RSSM_READ_NVFP4:
+        codes = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(codes.shape[:-1] + (-1,))
+        want_codes, want_scales = oc.nvfp4_quantize(layer.ckpt.cpu().numpy())
+        deq = oc.nvfp4_dequantize(want_codes, want_scales)
+        np.testing.assert_array_equal(scales, want_scales, err_msg=what)
+    else:
+        want_codes, want_scales = oc.fp8_row_quantize(layer.ckpt.cpu().numpy())
+        deq = oc.fp8_row_dequantize(want_codes, want_scales)
+        np.testing.assert_array_equal(scales.view(np.uint32), want_scales.view(np.uint32), err_msg=what)
+    np.testing.assert_array_equal(codes, want_codes, err_msg=what)
+    return np.asarray(deq, dtype=np.float64)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_read_copy_view_through_folds(fmt):
+    """Decodes (the read-copy decode kernel) and verify rounds with seeded
+    acceptance, rows folding at different calls: after the window fills, and
+    before a token or drafts that do not fit (a pre-fold, after which the reads
+    see the copy the fold just wrote).  Every output equals the recurrence from
+    the copy's values R; the copy is the quantised fp32 checkpoint after every
+    call, and after each fold that checkpoint equals the exact state S."""
+    B, L, k = 3, 6, 3
+    shape = si.Mamba2Layer(batch=B, nheads=16, headdim=64, dstate=128, ngroups=2, window=L, dtype="bf16",
+                           state_std=0.1, max_draft=k)
+    layer, A, D, h0 = m2_layer(shape, read_fmt=fmt)
+    S = h0.double().numpy()
+    R = _read_view(layer, fmt, "copy at creation")
+    book = ob.WindowBook(B, L, int(layer.layout.cap))
+    y = torch.empty(B, 16, 64, device=DEV)
+    yk = torch.empty(B, k, 16, 64, device=DEV)
+    rows = lambda m: np.asarray(m, dtype=bool)[:, None, None, None]
+    pre_seen = post_seen = 0
+    for i, op in enumerate("ddvdvddvvdddvdvddvd"):
+        if op == "d":
+            tok = si.mamba2_tokens(shape, 100 + i, seed=7)
+            plan = book.decode()
+            layer.decode_step(dev_inputs(tok, M2_KEYS), y)
+            pre, post = [p[1] for p in plan], [p[3] for p in plan]
+            C = _read_view(layer, fmt, f"copy after call {i}")
+            R_next, want = _oracle_step(np.where(rows(pre), C, R), tok, A, D)
+            assert_close(y.cpu(), want, TOL["bf16"], f"{fmt} decode {i}: outputs from the copy")
+            S_next, _ = _oracle_step(S, tok, A, D)
+            for b in range(B):
+                if post[b]:
+                    assert_close(layer.ckpt[b].cpu(), S_next[b], TOL["f32"], f"decode {i} row {b}: folded checkpoint")
+                elif pre[b]:
+                    assert_close(layer.ckpt[b].cpu(), S[b], TOL["f32"], f"decode {i} row {b}: pre-folded checkpoint")
+            pre_seen += sum(pre)
+            post_seen += sum(post)
+            R = np.where(rows(post), C, R_next)
+            S = S_next
+        else:
+            drafts = si.mamba2_drafts(shape, i, k, seed=7)
+            acc = si.accept_counts(B, i, k, seed=5)   # (this seed leaves some rows full before a decode)
+            plan = book.verify(k)
+            layer.verify(k, dev_inputs(drafts, M2_KEYS), yk)
+            pre = [p[1] for p in plan]
+            C = _read_view(layer, fmt, f"copy after call {i}")
+            want, R_next = osp.mamba2_round(np.where(rows(pre), C, R), tok64(drafts), acc.numpy(), A, D)
+            assert_close(yk.cpu(), want, TOL["bf16"], f"{fmt} verify {i}: outputs from the copy")
+            for b in range(B):
+                if pre[b]:
+                    assert_close(layer.ckpt[b].cpu(), S[b], TOL["f32"], f"verify {i} row {b}: pre-folded checkpoint")
+            _, S = osp.mamba2_round(S, tok64(drafts), acc.numpy(), A, D)
+            n_reject = (k - acc).to(torch.int32)
+            layer.rollback(n_reject.to(DEV))
+            book.rollback(n_reject.tolist())
+            R = R_next
+        assert _bk(layer) == [list(x) for x in book.snapshot()], f"pointers after call {i}"
+    assert post_seen > 0 and pre_seen > 0, (post_seen, pre_seen)
+    layer.flush()
+    book.flush()
+    assert_close(layer.ckpt.cpu(), S, TOL["f32"], "checkpoint after the final flush")
+    _read_view(layer, fmt, "copy after the final flush")
+    assert layer.get_status() == 0
