@@ -6,6 +6,8 @@
 #include <new>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rssm_internal.h"
 #include "rssm_kda.h"
 
@@ -21,6 +23,15 @@ struct rssm_handle {
 };
 
 namespace {
+
+// An NVTX range named after the rssm_* call it covers, open for the call's
+// duration (a no-op unless a profiler that collects NVTX ranges is attached).
+struct CallRange {
+  explicit CallRange(const char *name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange &) = delete;
+  CallRange &operator=(const CallRange &) = delete;
+};
 
 thread_local std::string g_err;
 std::atomic<uint64_t> g_launches{0};
@@ -240,6 +251,7 @@ extern "C" {
 
 int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes, size_t *buf_bytes,
                         size_t *read_copy_bytes, size_t *meta_bytes, rssm_layout *layout) {
+  const CallRange call_range(__func__);
   int rc = validate_desc(desc);
   if (rc) return rc;
   if (!ckpt_bytes || !buf_bytes || !read_copy_bytes || !meta_bytes)
@@ -251,6 +263,7 @@ int rssm_workspace_size(const rssm_layer_desc *desc, size_t *ckpt_bytes, size_t 
 
 int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev, void *read_copy_dev,
                 void *meta_dev, rssm_handle **out) {
+  const CallRange call_range(__func__);
   int rc = validate_desc(desc);
   if (rc) return rc;
   if (!out) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
@@ -278,11 +291,13 @@ int rssm_create(const rssm_layer_desc *desc, void *ckpt_dev, void *buf_dev, void
 }
 
 int rssm_destroy(rssm_handle *h) {
+  const CallRange call_range(__func__);
   delete h;
   return ok();
 }
 
 int rssm_reset(rssm_handle *h, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   cudaError_t e = cudaMemsetAsync(h->meta, 0, h->meta_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(meta)");
@@ -296,6 +311,7 @@ int rssm_reset(rssm_handle *h, rssm_stream_t stream) {
 }
 
 int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.kind == RSSM_MAMBA2 && (!A_dev || !D_dev))
     return fail(RSSM_ERR_INVALID_ARG, "A and D must not be NULL");
@@ -305,6 +321,7 @@ int rssm_set_params(rssm_handle *h, const float *A_dev, const float *D_dev) {
 }
 
 int rssm_set_wait_limit(rssm_handle *h, long long cycles) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (cycles < 0) return fail(RSSM_ERR_INVALID_ARG, "wait limit must be >= 0 (0 = default)");
   h->wait_limit = cycles == 0 ? rssm::kDefaultWaitLimit : cycles;
@@ -312,6 +329,7 @@ int rssm_set_wait_limit(rssm_handle *h, long long cycles) {
 }
 
 int rssm_arm_timeout_test(rssm_handle *h) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.kind == RSSM_KDA && rssm::kda_fold_scratch_bytes(h->d) == 0)
     return fail(RSSM_ERR_UNSUPPORTED, "only the KDA decode serving kernel (bf16 inputs) has waits to run out");
@@ -320,6 +338,7 @@ int rssm_arm_timeout_test(rssm_handle *h) {
 }
 
 int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   int rc = check_inputs(h, in, out_dev);
   if (rc) return rc;
@@ -327,6 +346,7 @@ int rssm_decode_step(rssm_handle *h, const void *const *in, void *out_dev, rssm_
 }
 
 int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.max_draft < 1) return fail(RSSM_ERR_STATE, "handle was created with max_draft = 0");
   if (k < 1 || k > h->d.max_draft)
@@ -337,6 +357,7 @@ int rssm_verify(rssm_handle *h, int k, const void *const *in, void *out_dev, rss
 }
 
 int rssm_rollback(rssm_handle *h, const int32_t *n_reject_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!n_reject_dev) return fail(RSSM_ERR_INVALID_ARG, "n_reject is NULL");
   rssm::StepArgs a = step_args(h, rssm::kVerify, 0);
@@ -347,6 +368,7 @@ int rssm_rollback(rssm_handle *h, const int32_t *n_reject_dev, rssm_stream_t str
 }
 
 int rssm_flush(rssm_handle *h, const int32_t *row_mask_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.kind == RSSM_MAMBA2 && (!h->A || !h->D))
     return fail(RSSM_ERR_STATE, "Mamba-2 parameters not set (rssm_set_params)");
@@ -354,6 +376,7 @@ int rssm_flush(rssm_handle *h, const int32_t *row_mask_dev, rssm_stream_t stream
 }
 
 int rssm_quantize_read_copy(rssm_handle *h, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!h->rc) return fail(RSSM_ERR_STATE, "handle has no read copy (read_fmt = RSSM_READ_FP32)");
   rssm::QuantArgs q;
@@ -370,6 +393,7 @@ int rssm_quantize_read_copy(rssm_handle *h, rssm_stream_t stream) {
 
 int rssm_conventional_step(rssm_handle *h, const float *state_in_dev, float *state_out_dev,
                            const void *const *in, void *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!state_in_dev || !state_out_dev) return fail(RSSM_ERR_INVALID_ARG, "state pointers must not be NULL");
   if (!aligned(state_in_dev, 16) || !aligned(state_out_dev, 16))
@@ -400,6 +424,7 @@ int rssm_conventional_step(rssm_handle *h, const float *state_in_dev, float *sta
 int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev, const void *scales_in_dev,
                                      void *codes_out_dev, void *scales_out_dev, const void *const *in,
                                      void *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.read_fmt == RSSM_READ_FP32)
     return fail(RSSM_ERR_STATE, "the layer has no low-precision format (read_fmt is RSSM_READ_FP32)");
@@ -436,6 +461,7 @@ int rssm_conventional_step_quantized(rssm_handle *h, const void *codes_in_dev, c
 }
 
 int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!parent_dev) return fail(RSSM_ERR_INVALID_ARG, "parent is NULL");
   if (!h->d.branching) return fail(RSSM_ERR_STATE, "handle was created with branching = 0");
@@ -484,6 +510,7 @@ int rssm_branch(rssm_handle *h, const int32_t *parent_dev, rssm_stream_t stream)
 }
 
 int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!keep_dev) return fail(RSSM_ERR_INVALID_ARG, "keep is NULL");
   rssm::StepArgs a = step_args(h, rssm::kDecode, 0);
@@ -494,6 +521,7 @@ int rssm_restore(rssm_handle *h, const int32_t *keep_dev, rssm_stream_t stream) 
 }
 
 int rssm_get_slots(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!out_dev) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
   if (!h->d.branching) return fail(RSSM_ERR_STATE, "handle was created with branching = 0");
@@ -523,6 +551,7 @@ int state_pieces(const rssm_handle *h, Piece (&p)[4]) {
 }  // namespace
 
 int rssm_state_bytes(rssm_handle *h, size_t *bytes) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!bytes) return fail(RSSM_ERR_INVALID_ARG, "bytes is NULL");
   Piece p[4];
@@ -552,14 +581,17 @@ static int copy_state(rssm_handle *h, uint8_t *host, size_t bytes, bool to_host,
 }
 
 int rssm_export_state(rssm_handle *h, void *host_dst, size_t bytes, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   return copy_state(h, static_cast<uint8_t *>(host_dst), bytes, true, (cudaStream_t)stream);
 }
 
 int rssm_import_state(rssm_handle *h, const void *host_src, size_t bytes, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   return copy_state(h, static_cast<uint8_t *>(const_cast<void *>(host_src)), bytes, false, (cudaStream_t)stream);
 }
 
 int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!out_dev) return fail(RSSM_ERR_INVALID_ARG, "out is NULL");
   rssm::StepArgs a = step_args(h, rssm::kDecode, 0);
@@ -571,6 +603,7 @@ int rssm_get_bookkeeping(rssm_handle *h, int32_t *out_dev, rssm_stream_t stream)
 }
 
 int rssm_get_lengths(rssm_handle *h, int32_t *len_dev, int32_t *pending_dev, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!len_dev || !pending_dev) return fail(RSSM_ERR_INVALID_ARG, "len or pending is NULL");
   const size_t n = sizeof(int32_t) * (size_t)h->d.batch;
@@ -584,6 +617,7 @@ int rssm_get_lengths(rssm_handle *h, int32_t *len_dev, int32_t *pending_dev, rss
 }
 
 int rssm_get_status(rssm_handle *h, uint32_t *bits, int clear, rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (!bits) return fail(RSSM_ERR_INVALID_ARG, "bits is NULL");
   uint32_t *dev = reinterpret_cast<uint32_t *>(h->meta + h->lay.meta_status_off);
@@ -641,6 +675,7 @@ int static_arrivals_for_current_device(int32_t **out) {
 
 extern "C" int rssm_decode_step_static_scratch(rssm_handle *h, const void *const *in, void *out_dev,
                                                rssm_stream_t stream) {
+  const CallRange call_range(__func__);
   if (!h) return fail(RSSM_ERR_INVALID_ARG, "handle is NULL");
   if (h->d.batch > RSSM_STATIC_SCRATCH_MAX_BATCH)
     return fail(RSSM_ERR_INVALID_ARG,

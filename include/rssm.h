@@ -47,6 +47,8 @@
  *     pending) leave that row untouched -- no output written, no state or
  *     pointer moved -- and set a sticky bit in the device status word.
  *   - Row-major layouts; the last index is contiguous.
+ *   - Tracing: every call that returns an int is an NVTX range named after
+ *     the call (a no-op unless a profiler collecting NVTX ranges is attached).
  */
 #ifndef RSSM_H
 #define RSSM_H
