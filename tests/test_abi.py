@@ -230,6 +230,23 @@ def test_kda_descriptor_and_layout():
         assert L.rssm_arm_timeout_test(h) == rssm.RSSM_ERR_UNSUPPORTED
     finally:
         L.rssm_destroy(h)
+    # a read copy: the create call needs its buffer; the serving kernel (fp32 reads only)
+    # allocates no fold scratch, so the decode kernel has no waits to arm; the stored
+    # low-precision state baseline is Mamba-2 / GDN only
+    d_ = _desc(**dict(base, read_fmt=rssm.RSSM_READ_NVFP4))
+    code, (ck4, buf4, rc4, meta4), lay4 = _sizes(d_)
+    assert lay4.fold_scratch_off == 0
+    assert L.rssm_create(C.byref(d_), fake, fake, None, fake, C.byref(h)) == rssm.RSSM_ERR_INVALID_ARG
+    assert L.rssm_create(C.byref(d_), fake, fake, fake, fake, C.byref(h)) == rssm.RSSM_OK
+    try:
+        assert L.rssm_arm_timeout_test(h) == rssm.RSSM_ERR_UNSUPPORTED
+        n = C.c_size_t()
+        assert L.rssm_state_bytes(h, C.byref(n)) == rssm.RSSM_OK and n.value == ck4 + rc4 + buf4 + meta4
+        ins = (C.c_void_p * 5)(fake, fake, fake, fake, fake)
+        assert L.rssm_conventional_step_quantized(h, fake, fake, fake, fake, ins, fake, None) == \
+            rssm.RSSM_ERR_UNSUPPORTED
+    finally:
+        L.rssm_destroy(h)
 
 
 def test_state_io_checks_sizes():
